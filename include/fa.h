@@ -1,0 +1,124 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) FlashAttention forward library (libfa_sm100.so).
+ *
+ * What is computed
+ * ----------------
+ * Exact scaled dot-product attention, one tile of keys at a time, with the online
+ * softmax: per query row a running maximum m and sum l are kept, and the output
+ * accumulator is rescaled by exp(m_old - m_new) whenever the maximum grows, so the
+ * N x N score matrix never reaches device memory.  Sources:
+ *   - "Module 16: Efficient and Long Attention" (transformers-and-math), section 16.2,
+ *     the online softmax and the two-block merge identities; "the result is exactly
+ *     standard attention, up to rounding";
+ *   - "Online Softmax Without the Attention Matrix" (notebook): the tile recurrence
+ *     new max -> correction exp(old - new) -> rescaled sums;
+ *   - oxios flash_attention.rs, FlashAttention::attention: queries / keys / values ->
+ *     output, scale 1/(temperature * sqrt(d)), the -inf guard on the first rescale.
+ *
+ * For every batch b, query head hq and query row i (0 <= i < N), with the key/value
+ * head kv = hq / (Hq / Hkv) (contiguous groups for grouped-query attention):
+ *   s_j   = scale * <q[b,hq,i,:], k[b,kv,j,:]>                       0 <= j < N
+ *   s_j   = softcap * tanh(s_j / softcap)        if softcap > 0     (Module 16, 16.5)
+ *   s_j   = -inf   if causal and j > i                              (Module 16, 16.2)
+ *   s_j   = -inf   if window > 0 and i - j >= window                (Module 16, 16.3:
+ *                                                                    the W most recent
+ *                                                                    tokens, self included)
+ *   o[b,hq,i,:] = sum_j softmax(s)_j * v[b,kv,j,:]
+ *   lse[b,hq,i] = ln sum_j exp(s_j)        (natural log of the final, masked scores)
+ *
+ * Layout and ownership
+ * --------------------
+ *   q, o : [B, Hq,  N, d] row-major, contiguous;  k, v : [B, Hkv, N, d];  lse : [B, Hq, N].
+ *   All pointers are DEVICE pointers owned by the caller.  q, k, v and o must be 16-byte
+ *   aligned, lse 4-byte aligned.  The library allocates no device memory, keeps no
+ *   per-call state and does not synchronise: work is queued on `stream` (a
+ *   cudaStream_t; NULL is the legacy default stream) and the outputs are valid once
+ *   that stream has been synchronised.  Calls are asynchronous, so launch errors that
+ *   only show later (and device-side wait timeouts) are reported by fa_check_status().
+ *
+ * Errors
+ * ------
+ * Every entry point returns FA_OK (0) or one of the negative codes below and writes
+ * nothing when it rejects its arguments.  B == 0 or N == 0 (or Hq == 0) is a valid
+ * empty problem: it returns FA_OK and touches no memory (oxios returns an empty result
+ * for empty input).  lse == NULL skips the log-sum-exp output.
+ */
+#ifndef FA_SM100_H_
+#define FA_SM100_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FA_OK 0
+#define FA_ERR_NULL_PTR (-1)    /* q, k, v or o is NULL (and the problem is not empty)   */
+#define FA_ERR_BAD_SHAPE (-2)   /* a size < 0, Hkv == 0 or Hq % Hkv != 0, size overflow  */
+#define FA_ERR_UNSUPPORTED (-3) /* head dim / mask combination this path does not cover,
+                                   or the current device is not sm_100                  */
+#define FA_ERR_ALIGN (-4)       /* a pointer breaks the alignment rule above             */
+#define FA_ERR_BAD_ARG (-5)     /* scale not finite or <= 0, softcap not finite          */
+#define FA_ERR_CUDA (-6)        /* a CUDA runtime/driver call failed: fa_last_cuda_error */
+#define FA_ERR_TIMEOUT (-7)     /* a device-side wait exceeded its limit (see below)     */
+
+/*
+ * fa_fwd -- bf16 attention forward on the tensor cores (tcgen05 + TMA + TMEM).
+ *   q, k, v, o : __nv_bfloat16 device arrays (layout above); lse : float or NULL.
+ *   B, Hq, Hkv, N : batch, query heads, key/value heads, sequence length (queries and
+ *                   keys share N: self-attention).
+ *   d        : head dimension, 64 or 128.
+ *   scale    : multiplier of q.k (e.g. 1/sqrt(d); a softmax temperature T folds in as
+ *              1/(T sqrt(d))), finite and > 0.
+ *   causal   : non-zero masks keys j > i.
+ *   window   : > 0 keeps only keys with i - j < window (requires causal); <= 0 is off.
+ *   softcap  : > 0 applies softcap * tanh(s / softcap) after the scale; <= 0 is off.
+ *   stream   : cudaStream_t (NULL = legacy default stream).
+ * Precision: bf16 operands, fp32 accumulation of Q.K^T and P.V, probabilities P
+ * rounded to bf16 (round-to-nearest-even) for the P.V product, running sum l in fp32,
+ * output rounded to bf16 (RNE), lse in fp32.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+           int N, int d, float scale, int causal, int window, float softcap, void* stream);
+
+/*
+ * fa_fwd_f32 -- the same operation in fp32 on the CUDA cores (FFMA, no TF32), for
+ * small head dimensions: 1 <= d <= 128.  Same arguments as fa_fwd with float q, k, v,
+ * o.  Pointers need 4-byte alignment.  Scores, the online-softmax state and the
+ * accumulator are fp32; exponentials use the accurate expf.
+ * Source of the workload it was built for: nx_flashattn_scale.nx (n = 64, d = 32,
+ * f32 streaming attention checked against a direct softmax).
+ */
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Hq,
+               int Hkv, int N, int d, float scale, int causal, int window, float softcap, void* stream);
+
+/*
+ * fa_check_status -- synchronise `stream`, then report (and clear) the device status
+ * word that kernels of this library set when one of their bounded waits ran out
+ * (FA_ERR_TIMEOUT) on the current device, or a pending CUDA error (FA_ERR_CUDA).
+ * Returns FA_OK when neither happened.
+ */
+int fa_check_status(void* stream);
+
+/*
+ * fa_selftest_wait_timeout -- failure-detection self-test: launches one tiny kernel
+ * whose single wait (the same bounded mbarrier wait the attention kernels use) is on a
+ * barrier that nothing ever arrives at, with a limit of `timeout_us` microseconds
+ * (1..1000000).  The wait gives up, the kernel records FA_ERR_TIMEOUT and exits.
+ * Synchronises `stream` and returns what fa_check_status() reports (FA_ERR_TIMEOUT
+ * when the mechanism works); the device stays usable.
+ */
+int fa_selftest_wait_timeout(unsigned timeout_us, void* stream);
+
+/* fa_strerror -- static description of an FA_* code. */
+const char* fa_strerror(int code);
+
+/* fa_last_cuda_error -- the cudaError_t of the last failed CUDA call on this thread. */
+int fa_last_cuda_error(void);
+
+/* fa_version -- library ABI version (major * 100 + minor). */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H_ */

@@ -1,0 +1,287 @@
+// fa_api.cu -- host side of the C ABI declared in include/fa.h: argument checks, TMA
+// descriptors, kernel selection and launch.  Everything here is plain pointers and sizes;
+// no framework types cross the boundary.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_fwd_f32.cuh"
+#include "fa_fwd_tc.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return FA_ERR_CUDA;
+}
+
+// Default limit of one device-side wait.  A healthy wait ends in microseconds; the
+// limit only has to separate "slow" from "never".
+constexpr unsigned long long kWaitLimitNs = 2ull * 1000 * 1000 * 1000;
+
+constexpr int kMaxDevices = 64;
+
+// Per-device facts checked once: compute capability and kernel attributes.
+struct DeviceState {
+  std::once_flag once;
+  int status = FA_OK;
+};
+DeviceState g_dev[kMaxDevices];
+
+int current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (*dev < 0 || *dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+int prepare_device(int dev) {
+  DeviceState& st = g_dev[dev];
+  std::call_once(st.once, [&] {
+    cudaDeviceProp prop;
+    cudaError_t e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) {
+      st.status = cuda_fail(e);
+      return;
+    }
+    if (prop.major != 10 || prop.minor != 0) {  // built for sm_100a only
+      st.status = FA_ERR_UNSUPPORTED;
+      return;
+    }
+    e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::tc::Layout<128>::kSmemLaunch);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::tc::Layout<64>::kSmemLaunch);
+    // the fp32 path needs up to 4 * (32 d + 32 (d + 1) + 32 d) bytes = 49280 at d = 128
+    const int f32_smem = 64 * 1024;
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_fwd_f32_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, f32_smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_fwd_f32_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, f32_smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_fwd_f32_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, f32_smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_fwd_f32_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, f32_smem);
+    if (e != cudaSuccess) st.status = cuda_fail(e);
+  });
+  return st.status;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// [heads, N, d] bf16 tensor viewed as 3-D (d, N, heads); boxes of 64 columns x 128 rows
+// with 128-byte swizzle, which is the canonical K-major (Q, K) and MN-major (V) operand
+// layout of tcgen05.mma.  Rows past N read as zero.
+int make_map(CUtensorMap* map, const void* base, int heads, int N, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cuda_fail(cudaErrorNotSupported);
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem_strides,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return FA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Checks shared by both entry points.  Returns FA_OK, an error, or 1 for "empty problem".
+int check_common(const void* q, const void* k, const void* v, const void* o, int B, int Hq, int Hkv, int N, int d,
+                 float scale, int causal, int window, float softcap) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || N < 0 || d < 0) return FA_ERR_BAD_SHAPE;
+  if (Hkv == 0 || (Hq % Hkv) != 0) return FA_ERR_BAD_SHAPE;
+  if (!std::isfinite(scale) || !(scale > 0.f) || !std::isfinite(softcap)) return FA_ERR_BAD_ARG;
+  if (window > 0 && !causal) return FA_ERR_UNSUPPORTED;
+  // element counts must fit the kernels' index arithmetic
+  const long long rows = static_cast<long long>(B) * Hq * N;
+  if (rows > (1ll << 31) - 1 || static_cast<long long>(B) * Hq > (1ll << 31) - 1) return FA_ERR_BAD_SHAPE;
+  if (B == 0 || Hq == 0 || N == 0) return 1;
+  if (d == 0) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o) return FA_ERR_NULL_PTR;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+int fa_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* fa_strerror(int code) {
+  switch (code) {
+    case FA_OK: return "ok";
+    case FA_ERR_NULL_PTR: return "a required pointer is NULL";
+    case FA_ERR_BAD_SHAPE: return "bad shape (negative size, Hkv == 0, Hq % Hkv != 0 or size overflow)";
+    case FA_ERR_UNSUPPORTED: return "unsupported head dimension, mask combination or device";
+    case FA_ERR_ALIGN: return "pointer not aligned as required";
+    case FA_ERR_BAD_ARG: return "scale must be finite and > 0, softcap finite";
+    case FA_ERR_CUDA: return "CUDA call failed (see fa_last_cuda_error)";
+    case FA_ERR_TIMEOUT: return "a device-side wait exceeded its limit";
+    default: return "unknown error code";
+  }
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d,
+           float scale, int causal, int window, float softcap, void* stream) {
+  int rc = check_common(q, k, v, o, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4)))
+    return FA_ERR_ALIGN;
+  int dev;
+  if ((rc = current_device(&dev)) != FA_OK) return rc;
+  if ((rc = prepare_device(dev)) != FA_OK) return rc;
+
+  CUtensorMap mq, mk, mv;
+  if ((rc = make_map(&mq, q, B * Hq, N, d)) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * Hkv, N, d)) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * Hkv, N, d)) != FA_OK) return rc;
+
+  namespace tc = fa::tc;
+  tc::Params p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.n_qpairs = (N + tc::NQ * tc::BM - 1) / (tc::NQ * tc::BM);
+  p.causal = causal ? 1 : 0;
+  p.window = window > 0 ? window : 0;
+  p.scale_log2 = scale * tc::kLog2e;
+  p.use_softcap = softcap > 0.f ? 1 : 0;
+  p.cap_inner = softcap > 0.f ? scale / softcap : 0.f;
+  p.cap_outer = softcap > 0.f ? softcap * tc::kLog2e : 0.f;
+  p.timeout_ns = kWaitLimitNs;
+
+  const long long grid = static_cast<long long>(B) * Hq * p.n_qpairs;
+  if (grid > 0x7fffffffll) return FA_ERR_BAD_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128) {
+    tc::fa_fwd_tc_kernel<128><<<static_cast<unsigned>(grid), tc::kThreads, tc::Layout<128>::kSmemLaunch, s>>>(
+        mq, mk, mv, p);
+  } else {
+    tc::fa_fwd_tc_kernel<64><<<static_cast<unsigned>(grid), tc::kThreads, tc::Layout<64>::kSmemLaunch, s>>>(
+        mq, mk, mv, p);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
+}
+
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Hq, int Hkv, int N,
+               int d, float scale, int causal, int window, float softcap, void* stream) {
+  int rc = check_common(q, k, v, o, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (d < 1 || d > fa::f32path::kMaxD) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(o, 4) || (lse && !aligned(lse, 4)))
+    return FA_ERR_ALIGN;
+  int dev;
+  if ((rc = current_device(&dev)) != FA_OK) return rc;
+  if ((rc = prepare_device(dev)) != FA_OK) return rc;
+
+  namespace f = fa::f32path;
+  const int q_blocks = (N + f::kRows - 1) / f::kRows;
+  const long long grid = static_cast<long long>(B) * Hq * q_blocks;
+  if (grid > 0x7fffffffll) return FA_ERR_BAD_SHAPE;
+  const size_t smem = sizeof(float) * (static_cast<size_t>(f::kRows) * d + static_cast<size_t>(f::kKeys) * (d + 1) +
+                                       static_cast<size_t>(f::kKeys) * d);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float cap = softcap > 0.f ? softcap : 0.f;
+  const int win = window > 0 ? window : 0;
+  const int dpl = (d + 31) / 32;
+  const unsigned g = static_cast<unsigned>(grid);
+  switch (dpl) {
+    case 1: fa::fa_fwd_f32_kernel<1><<<g, f::kThreads, smem, s>>>(q, k, v, o, lse, Hq, Hkv, N, d, scale, causal, win, cap, q_blocks); break;
+    case 2: fa::fa_fwd_f32_kernel<2><<<g, f::kThreads, smem, s>>>(q, k, v, o, lse, Hq, Hkv, N, d, scale, causal, win, cap, q_blocks); break;
+    case 3: fa::fa_fwd_f32_kernel<3><<<g, f::kThreads, smem, s>>>(q, k, v, o, lse, Hq, Hkv, N, d, scale, causal, win, cap, q_blocks); break;
+    default: fa::fa_fwd_f32_kernel<4><<<g, f::kThreads, smem, s>>>(q, k, v, o, lse, Hq, Hkv, N, d, scale, causal, win, cap, q_blocks); break;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// status word and the failure-detection self-test
+// ---------------------------------------------------------------------------------
+namespace {
+
+__global__ void fa_wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    fa::mbar_init(&bar, 1);
+    abort_flag = 0;
+    fa::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // nothing ever arrives on `bar`: the bounded wait must give up by itself
+    fa::mbar_wait(&bar, 0, fa::WaitCtl{&abort_flag, limit_ns});
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_check_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  int st = 0;
+  e = cudaMemcpyFromSymbol(&st, fa::g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (st != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(fa::g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return st;
+  }
+  return FA_OK;
+}
+
+int fa_selftest_wait_timeout(unsigned timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return FA_ERR_BAD_ARG;
+  int dev, rc;
+  if ((rc = current_device(&dev)) != FA_OK) return rc;
+  if ((rc = prepare_device(dev)) != FA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  fa_wait_selftest_kernel<<<1, 32, 0, s>>>(static_cast<unsigned long long>(timeout_us) * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return fa_check_status(stream);
+}
+
+}  // extern "C"

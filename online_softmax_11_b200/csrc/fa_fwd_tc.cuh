@@ -1,0 +1,489 @@
+// fa_fwd_tc.cuh -- bf16 attention forward on the Blackwell tensor cores (sm_100a).
+//
+// One CTA owns two 128-row query tiles (Q0, Q1) of one (batch, query head) and streams
+// the 128-key K/V tiles they need through shared memory.  Per key tile j and query
+// tile i it computes ("Module 16: Efficient and Long Attention", 16.1 and 16.2):
+//   S_i   = Q_i K_j^T                          tcgen05.mma, A and B from shared memory,
+//                                              fp32 accumulator in tensor memory (TMEM)
+//   s    <- scale * s, soft-cap, mask          (16.5 soft-cap; 16.2 "Measured": the mask
+//                                              uses positions in the full sequence)
+//   m_new = max(m, rowmax s)                   one query row per thread: row max and sum
+//   P     = exp(s - m), l = alpha l + sum P    are thread-local, P rounded to bf16 and
+//                                              written back into TMEM over S_i
+//   O_i   = alpha O_i + P V_j                  tcgen05.mma, A = P from TMEM, B = V from
+//                                              shared memory (MN-major, no transpose)
+// and finally O_i / l (bf16) and LSE = m + ln l (fp32), each written to HBM once.
+// The score matrix never leaves the SM.
+//
+// Roles (320 threads = 10 warps):
+//   warps 0-3  softmax warpgroup for Q0 (thread t owns TMEM lane t = query row t)
+//   warps 4-7  softmax warpgroup for Q1
+//   warp  8    TMA producer: Q0/Q1 once, then K_j, V_j into a ring of shared-memory slots
+//   warp  9    MMA issuer (one thread) and owner of the TMEM allocation
+// The two query tiles ping-pong: while one warpgroup exponentiates S_0, the tensor core
+// computes P_1 V and S_1 for the other, so the MMA pipe and the exponential units
+// overlap.
+//
+// Online-softmax details:
+//   * Scores are handled in log2 units, u = s * scale * log2(e), so P = exp2(u - m) is one
+//     FFMA plus one ex2 per score.
+//   * Lazy rescaling: the running maximum used for P only moves when the row maximum
+//     grows by more than kRescaleLog2 (2^8); P then stays <= 256, and O and l always share
+//     the same (possibly stale) reference, so the result is still exact up to rounding
+//     (Module 16, 16.2: the max subtraction is about range, not correctness).  When it
+//     moves, the row of O in TMEM is multiplied by alpha = exp2(m_old - m_new) before the
+//     next P V product is issued.
+//   * A row whose maximum is still -inf uses 0 as its reference, so masked scores give
+//     P = 0 and never NaN; alpha is 0 in that case (the guard of oxios'
+//     FlashAttention::attention for the first rescale).
+//
+// Every wait is bounded (see mbar_wait): a lost phase turns into FA_ERR_TIMEOUT in the
+// device status word and an orderly exit, never a hang.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+namespace tc {
+
+constexpr int BM = 128;                       // query rows per Q tile (= TMEM lanes)
+constexpr int BN = 128;                       // keys per K/V tile
+constexpr int NQ = 2;                         // Q tiles per CTA
+constexpr int kSoftmaxWarps = 4 * NQ;
+constexpr int kLoadWarp = kSoftmaxWarps;      // warp 8
+constexpr int kMmaWarp = kSoftmaxWarps + 1;   // warp 9
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+constexpr int kTmemCols = 512;                // S0 | S1 | O0 | O1, 128 columns each
+constexpr float kRescaleLog2 = 8.0f;          // lazy-rescale threshold (log2 units)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D>
+struct Layout {
+  static_assert(D == 64 || D == 128, "head dim 64 or 128");
+  static constexpr int kHalves = D / 64;               // 64-column (128-byte) slabs per row
+  static constexpr int kHalfBytes = 128 * 128;         // one slab of a 128-row tile
+  static constexpr int kTileBytes = 128 * D * 2;       // a Q, K or V tile
+  static constexpr int kStages = D == 128 ? 4 : 8;     // K/V ring slots
+  static constexpr int kQOff = 0;
+  static constexpr int kRingOff = kQOff + NQ * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
+  // barriers: q_full | kv_full[S] | kv_empty[S] | s_full[NQ] | p_full[NQ] | o_full[NQ] | drain
+  static constexpr int kBarQFull = 0;
+  static constexpr int kBarKvFull = 1;
+  static constexpr int kBarKvEmpty = kBarKvFull + kStages;
+  static constexpr int kBarSFull = kBarKvEmpty + kStages;
+  static constexpr int kBarPFull = kBarSFull + NQ;
+  static constexpr int kBarOFull = kBarPFull + NQ;
+  static constexpr int kBarDrain = kBarOFull + NQ;
+  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // u32 tmem base, int abort flag
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kSmemAlloc = kBytes + 1024;         // slack for 1024-byte alignment
+  // TMEM columns: S_i at 128 i, O_i at 256 + 128 i
+  __device__ static constexpr uint32_t col_s(int i) { return static_cast<uint32_t>(i) * 128u; }
+  __device__ static constexpr uint32_t col_o(int i) { return 256u + static_cast<uint32_t>(i) * 128u; }
+  // The d = 64 variant must not share an SM with a second CTA (TMEM is fully allocated).
+  static constexpr int kSmemLaunch = kSmemAlloc > 120 * 1024 ? kSmemAlloc : 120 * 1024;
+};
+
+struct Params {
+  __nv_bfloat16* o;
+  float* lse;
+  int Hq, Hkv, N;
+  int n_qpairs;        // ceil(N / (NQ * BM)) query-tile pairs per head
+  int causal;
+  int window;          // <= 0: off
+  float scale_log2;    // scale * log2(e)
+  int use_softcap;
+  float cap_inner;     // scale / softcap
+  float cap_outer;     // softcap * log2(e)
+  unsigned long long timeout_ns;
+};
+
+// Accurate tanh for the soft-cap: Taylor series about 0 through x^11 for |x| < 0.3
+// (truncation error below 1e-9), otherwise 1 - 2 / (exp(2|x|) + 1) with the sign of x.
+// The coefficients are the series of tanh: 1, -1/3, 2/15, -17/315, 62/2835, -1382/155925.
+__device__ __forceinline__ float tanh_cap(float x) {
+  const float ax = fabsf(x);
+  if (ax < 0.3f) {
+    const float x2 = x * x;
+    float p = -1382.0f / 155925.0f;
+    p = fmaf(p, x2, 62.0f / 2835.0f);
+    p = fmaf(p, x2, -17.0f / 315.0f);
+    p = fmaf(p, x2, 2.0f / 15.0f);
+    p = fmaf(p, x2, -1.0f / 3.0f);
+    return fmaf(p * x2, x, x);
+  }
+  const float e = ex2_approx(2.0f * kLog2e * ax);
+  const float t = 1.0f - __fdividef(2.0f, e + 1.0f);
+  return copysignf(t, x);
+}
+
+// Key-tile range of one query tile: [lo, hi) of 128-key tiles.
+struct TileRange {
+  int r0, r1;  // first / last query row (r1 < N)
+  int lo, hi;
+  bool active;
+};
+
+__device__ __forceinline__ TileRange tile_range(int r0, int N, int nkv, int causal, int window) {
+  TileRange t;
+  t.r0 = r0;
+  t.active = r0 < N;
+  t.r1 = min(N, r0 + BM) - 1;
+  t.lo = 0;
+  t.hi = nkv;
+  if (causal) t.hi = min(nkv, t.r1 / BN + 1);
+  if (window > 0) t.lo = max(0, t.r0 - window + 1) / BN;
+  if (!t.active) t.lo = t.hi = 0;
+  return t;
+}
+
+__device__ __forceinline__ bool participates(const TileRange& t, int j) { return t.active && j >= t.lo && j < t.hi; }
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  int* abort_flag = reinterpret_cast<int*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work tile: (batch*head, query-tile pair), longest rows first within a head
+  const int tile = blockIdx.x;
+  const int bh = tile / p.n_qpairs;
+  const int qp = p.n_qpairs - 1 - (tile - bh * p.n_qpairs);
+  const int b = bh / p.Hq;
+  const int hq = bh - b * p.Hq;
+  const int kvh = b * p.Hkv + hq / (p.Hq / p.Hkv);
+  const int N = p.N;
+  const int nkv = (N + BN - 1) / BN;
+  TileRange tr[NQ];
+#pragma unroll
+  for (int i = 0; i < NQ; ++i) tr[i] = tile_range(qp * NQ * BM + i * BM, N, nkv, p.causal, p.window);
+  int lo = tr[0].lo, hi = tr[0].hi;
+#pragma unroll
+  for (int i = 1; i < NQ; ++i)
+    if (tr[i].active) {
+      lo = min(lo, tr[i].lo);
+      hi = max(hi, tr[i].hi);
+    }
+  const int T = hi - lo;  // key tiles this CTA streams
+
+  // ---- set-up: barriers, abort flag, TMEM
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[L::kBarQFull], 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&bars[L::kBarKvFull + s], 1);
+      mbar_init(&bars[L::kBarKvEmpty + s], 1);
+    }
+    for (int i = 0; i < NQ; ++i) {
+      mbar_init(&bars[L::kBarSFull + i], 1);
+      mbar_init(&bars[L::kBarPFull + i], 128);
+      mbar_init(&bars[L::kBarOFull + i], 1);
+    }
+    mbar_init(&bars[L::kBarDrain], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_base_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_slot;
+  const WaitCtl ctl{abort_flag, p.timeout_ns};
+  const WaitCtl drain_ctl{abort_flag, 50ull * 1000 * 1000};
+
+  if (warp == kLoadWarp) {
+    // =========================== TMA producer ===========================
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      uint8_t* sQ = smem + L::kQOff;
+      uint32_t qbytes = 0;
+#pragma unroll
+      for (int i = 0; i < NQ; ++i) qbytes += tr[i].active ? L::kTileBytes : 0;
+      mbar_arrive_expect_tx(&bars[L::kBarQFull], qbytes);
+#pragma unroll
+      for (int i = 0; i < NQ; ++i)
+        if (tr[i].active)
+          for (int h = 0; h < L::kHalves; ++h)
+            tma_load_3d(sQ + i * L::kTileBytes + h * L::kHalfBytes, &tmQ, &bars[L::kBarQFull], h * 64, tr[i].r0,
+                        bh);
+      int issued = 0;  // loads issued into the ring (K and V alternate)
+      for (int n = 0; n < T && !*abort_flag; ++n) {
+        const int j = lo + n;
+        for (int which = 0; which < 2; ++which) {
+          const int s = issued % L::kStages;
+          const uint32_t fill = issued / L::kStages;
+          if (!mbar_wait(&bars[L::kBarKvEmpty + s], (fill & 1u) ^ 1u, ctl)) break;
+          uint8_t* dst = smem + L::kRingOff + s * L::kTileBytes;
+          mbar_arrive_expect_tx(&bars[L::kBarKvFull + s], L::kTileBytes);
+          for (int h = 0; h < L::kHalves; ++h)
+            tma_load_3d(dst + h * L::kHalfBytes, which ? &tmV : &tmK, &bars[L::kBarKvFull + s], h * 64, j * BN,
+                        kvh);
+          ++issued;
+        }
+      }
+      if (*abort_flag) {
+        // let the copies already in flight land before the CTA's shared memory goes away
+        int no_abort = 0;
+        const WaitCtl c{&no_abort, drain_ctl.limit_ns};
+        mbar_wait(&bars[L::kBarQFull], 0, c);
+        for (int k = issued - 1; k >= 0 && k >= issued - L::kStages; --k)
+          mbar_wait(&bars[L::kBarKvFull + (k % L::kStages)], (k / L::kStages) & 1u, c);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // =========================== MMA issuer ===========================
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);  // Q (K-major) x K (K-major)
+      constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, D, 0, 1);  // P (TMEM) x V (MN-major)
+      const uint32_t sQ = smem_addr(smem + L::kQOff);
+      const uint32_t sRing = smem_addr(smem + L::kRingOff);
+      bool ok = mbar_wait(&bars[L::kBarQFull], 0, ctl);
+      tc_fence_after();
+      uint32_t p_phase[NQ] = {};
+      uint32_t o_acc[NQ] = {};
+
+      auto issue_s = [&](int i, uint32_t k_tile) {
+        const uint32_t q_tile = sQ + i * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
+          mma_ss(tmem + L::col_s(i), smem_desc_sw128(q_tile + off, 16, 1024), smem_desc_sw128(k_tile + off, 16, 1024),
+                 kIdescS, kk > 0);
+        }
+        mma_commit(&bars[L::kBarSFull + i]);
+      };
+      auto issue_pv = [&](int i, uint32_t v_tile) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // A: 16 keys of P = 8 TMEM columns; B: 16 key rows of V (128 B each), the two
+          // 64-column slabs of V are L::kHalfBytes apart (leading byte offset)
+          mma_ts(tmem + L::col_o(i), tmem + L::col_s(i) + kk * 8,
+                 smem_desc_sw128(v_tile + kk * 16 * 128, L::kHalfBytes, 1024), kIdescPV, (kk > 0) || o_acc[i]);
+        }
+        o_acc[i] = 1;
+      };
+
+      for (int n = 0; ok && n <= T; ++n) {
+        const int j = lo + n;
+        const int kslot = (2 * n) % L::kStages;
+        const int vslot = (2 * n - 1) % L::kStages;
+        if (n < T) {
+          ok = mbar_wait(&bars[L::kBarKvFull + kslot], ((2 * n) / L::kStages) & 1u, ctl);
+          if (!ok) break;
+        }
+        if (n > 0) {
+          ok = mbar_wait(&bars[L::kBarKvFull + vslot], ((2 * n - 1) / L::kStages) & 1u, ctl);
+          if (!ok) break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+          if (n > 0 && participates(tr[i], j - 1)) {
+            ok = mbar_wait(&bars[L::kBarPFull + i], p_phase[i], ctl);
+            if (!ok) break;
+            p_phase[i] ^= 1u;
+            tc_fence_after();
+            issue_pv(i, sRing + vslot * L::kTileBytes);
+            if (!participates(tr[i], j)) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
+          }
+          if (n < T && participates(tr[i], j)) issue_s(i, sRing + kslot * L::kTileBytes);
+        }
+        if (!ok) break;
+        if (n < T) mma_commit(&bars[L::kBarKvEmpty + kslot]);
+        if (n > 0) mma_commit(&bars[L::kBarKvEmpty + vslot]);
+      }
+      // make sure nothing this thread issued is still running before TMEM is released
+      mma_commit(&bars[L::kBarDrain]);
+      int no_abort = 0;
+      mbar_wait(&bars[L::kBarDrain], 0, WaitCtl{&no_abort, drain_ctl.limit_ns});
+    }
+  } else {
+    // =========================== softmax warpgroups ===========================
+    const int i = warp >> 2;       // which Q tile
+    const int wq = warp & 3;       // TMEM lane quarter of this warp
+    const int trow = wq * 32 + lane;
+    const TileRange t = (i == 0) ? tr[0] : tr[1];
+    const int row = t.r0 + trow;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t colS = L::col_s(i);
+    const uint32_t colO = L::col_o(i);
+
+    float m = -CUDART_INF_F;  // running reference maximum (log2 units)
+    float l = 0.f;            // running sum of P (fp32) relative to m
+    float lr = 0.f;           // running sum of the bf16-rounded P relative to m
+    uint32_t s_phase = 0;
+    bool o_valid = false;
+    bool ok = true;
+
+    for (int n = 0; n < T && ok; ++n) {
+      const int j = lo + n;
+      if (!participates(t, j)) continue;
+      // tcgen05.ld/st are warp-collective: the whole warp leaves together or not at all
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[L::kBarSFull + i], s_phase, ctl));
+      if (!ok) break;
+      s_phase ^= 1u;
+      tc_fence_after();
+
+      float s[BN];
+      {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          tmem_ld32_wait(lane_base + colS + c * 32, r);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(r[x]);
+        }
+      }
+
+      const int k0 = j * BN;
+      const bool need_mask = (k0 + BN > N) || (p.causal && k0 + BN - 1 > t.r0) ||
+                             (p.window > 0 && t.r1 - k0 >= p.window);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const int key = k0 + c;
+          bool valid = key < N;
+          if (p.causal && key > row) valid = false;
+          if (p.window > 0 && row - key >= p.window) valid = false;
+          if (!valid) s[c] = -CUDART_INF_F;
+        }
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+      float m_tile;
+      if (p.use_softcap)
+        m_tile = (mx == -CUDART_INF_F) ? -CUDART_INF_F : p.cap_outer * tanh_cap(mx * p.cap_inner);
+      else
+        m_tile = mx * p.scale_log2;
+      const float m_new = fmaxf(m, m_tile);
+
+      if (!o_valid) {
+        m = m_new;  // nothing accumulated yet: adopt the maximum as is
+      } else {
+        const bool need = m_new > m + kRescaleLog2;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
+          if (need) {
+            l *= alpha;
+            lr *= alpha;
+            m = m_new;
+          }
+          uint32_t r[32];
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            tmem_ld32_wait(lane_base + colO + c * 32, r);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+            tmem_st32(lane_base + colO + c * 32, r);
+          }
+        }
+      }
+      const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
+
+      // P = exp2(u - m), 32 keys at a time: 16 packed bf16 pairs per chunk go straight to
+      // TMEM over the first 64 columns of S_i (two bf16 per 32-bit column).  Two sums are
+      // kept: l (fp32 P) for the log-sum-exp, and lr (the bf16-rounded P that the tensor
+      // core multiplies with V) to normalise O, so O is a weighted mean of V with exactly
+      // the weights the MMA used.
+      float lsum0 = 0.f, lsum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
+#pragma unroll
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        uint32_t packed[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const float a = s[cb * 32 + 2 * x];
+          const float bb = s[cb * 32 + 2 * x + 1];
+          float e0, e1;
+          if (p.use_softcap) {
+            e0 = ex2_approx(fmaf(tanh_cap(a * p.cap_inner), p.cap_outer, -m_use));
+            e1 = ex2_approx(fmaf(tanh_cap(bb * p.cap_inner), p.cap_outer, -m_use));
+            e0 = (a == -CUDART_INF_F) ? 0.f : e0;
+            e1 = (bb == -CUDART_INF_F) ? 0.f : e1;
+          } else {
+            e0 = ex2_approx(fmaf(a, p.scale_log2, -m_use));
+            e1 = ex2_approx(fmaf(bb, p.scale_log2, -m_use));
+          }
+          lsum0 += e0;
+          lsum1 += e1;
+          const uint32_t pk = pack_bf16x2(e0, e1);
+          rsum0 += __uint_as_float(pk << 16);
+          rsum1 += __uint_as_float(pk & 0xFFFF0000u);
+          packed[x] = pk;
+        }
+        tmem_st16(lane_base + colS + cb * 16, packed);
+      }
+      l += lsum0 + lsum1;
+      lr += rsum0 + rsum1;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars[L::kBarPFull + i]);
+      o_valid = true;
+    }
+
+    // ---- epilogue: O / l -> bf16, LSE = (m + log2 l) ln 2
+    if (ok && t.active) {
+      if (o_valid) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[L::kBarOFull + i], 0, ctl));
+        tc_fence_after();
+      }
+      if (ok) {
+        const float inv = lr > 0.f ? 1.0f / lr : 0.f;
+        __nv_bfloat16* orow = p.o + (static_cast<int64_t>(bh) * N + row) * D;
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          if (o_valid) {
+            tmem_ld32_wait(lane_base + colO + c * 32, r);
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) r[x] = 0u;
+          }
+          if (row < N) {
+            uint4 w[4];
+            uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+            for (int x = 0; x < 16; ++x)
+              wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * inv, __uint_as_float(r[2 * x + 1]) * inv);
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) dst[x] = w[x];
+          }
+        }
+        if (p.lse != nullptr && row < N)
+          p.lse[static_cast<int64_t>(bh) * N + row] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace tc
+}  // namespace fa
