@@ -1,0 +1,395 @@
+"""Attention-forward benchmark on B200: TFLOP/s and fraction of the dense BF16 peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one full attention forward of the workload (all of Q.K^T, masking, online
+softmax, P.V and the O / LSE write-back: one launch of the bf16 tensor-core kernel)
+over one batch of synthetic inputs already resident in HBM.  The headline workload is
+the causal B=8, H=32, N=4096, d=128 bf16 configuration.  FLOPs follow the convention
+4 B Hq N^2 d, halved for causal, 4 B Hq d (N W - W^2/2) for a causal window.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a device
+synchronisation, timed with CUDA events on the launching stream; for N > 1 (torchrun,
+one rank per GPU) every rank runs its own independent batch (weak scaling, no data-path
+collective) and the maximum time over ranks is used.  The inputs (768 MiB for the
+headline workload) are larger than the 126 MB L2, so no flush is needed between steps.
+
+Printed (rank 0, one JSON line): metric, value (whole-job TFLOP/s), roofline of the
+kernel against the measured peak, e2e (the same metric with pinned-host inputs copied
+in and outputs copied back inside the timed region), the fp64 CPU oracle timed on a
+bounded row sample (cpu_baseline), SM clocks sampled during the timed region, and the
+number of kernel launches in the timed region.
+
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only), as the reference
+arm of the comparison.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s on 1 B200 and % of dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+KERNEL_SOURCES = ["online_softmax_11_b200/csrc/fa_fwd_tc.cuh", "online_softmax_11_b200/csrc/sm100_ptx.cuh",
+                  "online_softmax_11_b200/csrc/fa_api.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    rec = d.get(workload)
+    if not rec or rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def closed_flops(w) -> float:
+    if w.window > 0:
+        return 4.0 * w.B * w.Hq * w.d * (w.N * w.window - w.window * w.window / 2.0)
+    f = 4.0 * w.B * w.Hq * w.N * w.N * w.d
+    return f / 2.0 if w.causal else f
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample_rows(w, n_rows: int, offset: int = 0):
+    """``n_rows`` flat row indices spread evenly over all heads and query positions (so the
+    causal / window work per row averages like the full workload), rotated by
+    ``offset``."""
+    total = w.B * w.Hq * w.N
+    stride = max(1, total // max(1, n_rows))
+    start = (offset * 7919) % stride
+    return np.arange(start, total, stride, dtype=np.int64)[:n_rows]
+
+
+def rows_flops(w, rows) -> float:
+    i = rows % w.N
+    lo = np.maximum(0, i - w.window + 1) if w.window > 0 else np.zeros_like(i)
+    hi = i if w.causal else np.full_like(i, w.N - 1)
+    return float(4.0 * w.d * np.maximum(0, hi - lo + 1).sum())
+
+
+def time_oracle(w, inputs, seconds: float, offset: int = 0):
+    """Time the fp64 oracle on a row sample sized to take about ``seconds``.
+    Returns (TFLOP/s, seconds, rows, threads)."""
+    import oracle
+    q, k, v = inputs
+    threads = oracle.host_threads()
+    probe = oracle_sample_rows(w, 64 * threads, offset)
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, rows=probe)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    n = int(max(threads, min(w.B * w.Hq * w.N, len(probe) * seconds / dt)))
+    rows = oracle_sample_rows(w, n, offset)
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, rows=rows)
+    dt = time.perf_counter() - t0
+    return rows_flops(w, rows) / dt / 1e12, dt, len(rows), threads
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def emit(obj):
+    print(json.dumps(obj), flush=True)
+
+
+def reference_arm(args, w):
+    """The fp64 CPU oracle as the reference implementation (rank 0 only)."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    inputs = workloads.make_inputs(w)
+    threads = oracle.host_threads()
+    budget = float(args.reference_seconds) / max(1, args.steps + args.warmup)
+    # per step: a row sample sized for `budget` seconds of oracle work
+    probe = oracle_sample_rows(w, 32 * threads)
+    t0 = time.perf_counter()
+    oracle.attention(*inputs, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, rows=probe)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    n_rows = int(max(threads, len(probe) * budget / dt))
+    total_flop = 0.0
+    total_s = 0.0
+    for step in range(args.warmup + args.steps):
+        rows = oracle_sample_rows(w, n_rows, step)
+        t0 = time.perf_counter()
+        oracle.attention(*inputs, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, rows=rows)
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            total_flop += rows_flops(w, rows)
+            total_s += dt
+    value = total_flop / total_s / 1e12
+    sample = (f"{n_rows} query rows per step spread over all {w.B * w.Hq} heads and positions of "
+              f"{w.name} (dense fp64 oracle; FLOPs counted as 4 d per unmasked pair)")
+    emit({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_s / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, **{k: v for k, v in w.describe().items() if k != "workload"}},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    })
+    return 0
+
+
+def gpu_arm(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import online_softmax_11_b200 as fa
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+    fa.load()
+
+    # each rank its own batch: seeds shifted by the rank (weak scaling, no data exchange)
+    seeds = tuple(s + 100 * rank for s in w.seeds())
+    q_h, k_h, v_h = workloads.make_inputs(w, seeds=seeds)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    def step():
+        rc = fa.fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.Hq, w.Hkv,
+                        w.N, w.d, w.scale, w.causal, w.window, w.softcap, sh, w.dtype)
+        if rc != 0:
+            raise fa.FAError(rc, fa.load(), "fa_fwd")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.check_status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    sampler = ClockSampler(local if ws > 1 else 0) if not args.no_clocks else None
+    if sampler is not None:
+        time.sleep(0.3)  # let the sampler start before the timed region
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if ws > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    clocks = sampler.stop() if sampler is not None else None
+    if fa.check_status() != 0:
+        raise RuntimeError("device status word set during the timed region")
+
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    flop_per_step = closed_flops(w)
+    per_launch_ms = elapsed_ms / args.steps
+    value = ws * flop_per_step * args.steps / (max_ms / 1e3) / 1e12
+
+    # ---- e2e: pinned host inputs -> device, forward, outputs -> pinned host, per step
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        op = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        lp = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            qd.copy_(qp, non_blocking=True)
+            kd.copy_(kp, non_blocking=True)
+            vd.copy_(vp, non_blocking=True)
+            fa.forward(qd, kd, vd, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, out=o,
+                       lse=lse, stream=stream)
+            op.copy_(o, non_blocking=True)
+            lp.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if ws > 1:
+            dist.barrier()
+        n_e2e = max(1, min(args.e2e_steps, args.steps))
+        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        es.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        ee.record(stream)
+        torch.cuda.synchronize(dev)
+        te = torch.tensor([es.elapsed_time(ee)], dtype=torch.float64, device=dev)
+        if ws > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = (q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size())
+        d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+        e2e = {"value": ws * flop_per_step * n_e2e / (float(te.item()) / 1e3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "ms_per_step": float(te.item()) / n_e2e}
+        del qp, kp, vp, op, lp, qd, kd, vd
+
+    # ---- CPU baseline: the fp64 oracle on a bounded row sample (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        tflops, secs, nrows, threads = time_oracle(w, (q_h, k_h, v_h), args.cpu_seconds)
+        cpu = {"value": tflops, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{nrows} query rows spread evenly over all {w.B * w.Hq} heads and positions of "
+                         f"{w.name}, {secs:.1f} s of fp64 work; FLOPs counted as 4 d per unmasked pair"}
+
+    peaks, peaks_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flop_per_step / (per_launch_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                "traffic": load_traffic(w.name), "peak_source": f"bf16_tflops (burst) of {peaks_src}",
+                "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                "kernel": f"fa_fwd_tc_kernel<{w.d}>", "algorithmic_flop_per_launch": flop_per_step}
+
+    if rank == 0:
+        cfg = {"workload": w.name, **{k: v for k, v in w.describe().items() if k != "workload"},
+               "flop_convention": "4 B Hq N^2 d, /2 causal; 4 B Hq d (N W - W^2/2) with a window",
+               "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{ws} (independent batches)"}
+        emit({
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": args.steps,
+        })
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=None, help="override B (profiling on a smaller case)")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=150.0,
+                    help="total oracle time budget of the reference arm")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args(argv)
+    w = workloads.WORKLOADS[args.workload]
+    if w.dtype != "bfloat16" and args.impl == "ours":
+        ap.error("the benchmark times the bf16 tensor-core path")
+    if args.batch is not None:
+        w = w.with_(B=args.batch)
+    ws, _, _ = dist_env()
+    if args.gpus != ws:
+        ap.error(f"--gpus {args.gpus} needs one process per GPU: launch with torchrun --nproc-per-node "
+                 f"{args.gpus} (WORLD_SIZE is {ws})")
+    if args.impl == "reference":
+        return reference_arm(args, w)
+    return gpu_arm(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

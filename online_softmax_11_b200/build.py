@@ -52,7 +52,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    res = subprocess.run(command(tmp, verbose), capture_output=True, text=True)
+    res = subprocess.run(command(tmp, verbose), capture_output=True, text=True, timeout=900)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
         raise RuntimeError("nvcc failed building libfa_sm100.so")

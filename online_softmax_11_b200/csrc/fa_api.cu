@@ -31,6 +31,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
   std::once_flag once;
   int status = FA_OK;
+  int num_sms = 0;
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -41,7 +42,7 @@ int current_device(int* dev) {
   return FA_OK;
 }
 
-int prepare_device(int dev) {
+int prepare_device(int dev, int* num_sms = nullptr) {
   DeviceState& st = g_dev[dev];
   std::call_once(st.once, [&] {
     cudaDeviceProp prop;
@@ -54,6 +55,8 @@ int prepare_device(int dev) {
       st.status = FA_ERR_UNSUPPORTED;
       return;
     }
+    st.num_sms = prop.multiProcessorCount;
+
     e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fa::tc::Layout<128>::kSmemLaunch);
     if (e == cudaSuccess)
@@ -71,6 +74,7 @@ int prepare_device(int dev) {
       e = cudaFuncSetAttribute(fa::fa_fwd_f32_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, f32_smem);
     if (e != cudaSuccess) st.status = cuda_fail(e);
   });
+  if (num_sms) *num_sms = st.num_sms;
   return st.status;
 }
 
@@ -156,9 +160,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4)))
     return FA_ERR_ALIGN;
-  int dev;
+  int dev, num_sms = 0;
   if ((rc = current_device(&dev)) != FA_OK) return rc;
-  if ((rc = prepare_device(dev)) != FA_OK) return rc;
+  if ((rc = prepare_device(dev, &num_sms)) != FA_OK) return rc;
 
   CUtensorMap mq, mk, mv;
   if ((rc = make_map(&mq, q, B * Hq, N, d)) != FA_OK) return rc;
@@ -172,7 +176,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.N = N;
-  p.n_qpairs = (N + tc::NQ * tc::BM - 1) / (tc::NQ * tc::BM);
+  p.n_bh = B * Hq;
+  p.n_qp = (N + tc::NQ * tc::BM - 1) / (tc::NQ * tc::BM);
+  p.units_per_head = (p.n_qp + 1) / 2;
   p.causal = causal ? 1 : 0;
   p.window = window > 0 ? window : 0;
   p.scale_log2 = scale * tc::kLog2e;
@@ -181,8 +187,11 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.cap_outer = softcap > 0.f ? softcap * tc::kLog2e : 0.f;
   p.timeout_ns = kWaitLimitNs;
 
-  const long long grid = static_cast<long long>(B) * Hq * p.n_qpairs;
-  if (grid > 0x7fffffffll) return FA_ERR_BAD_SHAPE;
+  const long long units = static_cast<long long>(B) * Hq * p.units_per_head;
+  if (units > 0x7fffffffll) return FA_ERR_BAD_SHAPE;
+  p.n_units = static_cast<int>(units);
+  // persistent: one CTA per SM (never more CTAs than units)
+  const long long grid = units < num_sms ? units : num_sms;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 128) {
     tc::fa_fwd_tc_kernel<128><<<static_cast<unsigned>(grid), tc::kThreads, tc::Layout<128>::kSmemLaunch, s>>>(

@@ -1,28 +1,38 @@
 // fa_fwd_tc.cuh -- bf16 attention forward on the Blackwell tensor cores (sm_100a).
 //
-// One CTA owns two 128-row query tiles (Q0, Q1) of one (batch, query head) and streams
-// the 128-key K/V tiles they need through shared memory.  Per key tile j and query
-// tile i it computes ("Module 16: Efficient and Long Attention", 16.1 and 16.2):
+// A work tile is two 128-row query tiles (Q0, Q1) of one (batch, query head).  For each
+// 128-key K/V tile j the work tile needs, and each query tile i, the CTA computes
+// ("Module 16: Efficient and Long Attention", 16.1 and 16.2):
 //   S_i   = Q_i K_j^T                          tcgen05.mma, A and B from shared memory,
 //                                              fp32 accumulator in tensor memory (TMEM)
 //   s    <- scale * s, soft-cap, mask          (16.5 soft-cap; 16.2 "Measured": the mask
 //                                              uses positions in the full sequence)
 //   m_new = max(m, rowmax s)                   one query row per thread: row max and sum
-//   P     = exp(s - m), l = alpha l + sum P    are thread-local, P rounded to bf16 and
+//   P     = exp(s - m), l = alpha l + sum P    are thread-local; P rounded to bf16 and
 //                                              written back into TMEM over S_i
 //   O_i   = alpha O_i + P V_j                  tcgen05.mma, A = P from TMEM, B = V from
 //                                              shared memory (MN-major, no transpose)
-// and finally O_i / l (bf16) and LSE = m + ln l (fp32), each written to HBM once.
-// The score matrix never leaves the SM.
+// and finally O_i / l (bf16) and LSE = m + ln l (fp32), each written to HBM once.  The
+// score matrix never leaves the SM.
 //
-// Roles (320 threads = 10 warps):
-//   warps 0-3  softmax warpgroup for Q0 (thread t owns TMEM lane t = query row t)
-//   warps 4-7  softmax warpgroup for Q1
-//   warp  8    TMA producer: Q0/Q1 once, then K_j, V_j into a ring of shared-memory slots
-//   warp  9    MMA issuer (one thread) and owner of the TMEM allocation
+// Persistent CTAs, one per SM.  The work tiles are grouped in units of two query-tile
+// pairs of one head, {q-pair n-1-p, q-pair p}; under a causal mask the two halves of a
+// unit cost (2(n-1-p)+1.5) + (2p+1.5) key tiles, the same for every unit, so a static
+// round-robin of units over the CTAs is balanced.  Units are numbered head-major, so the
+// CTAs running at the same time share the K/V of a few heads in L2.
+//
+// Roles (384 threads = 3 warpgroups):
+//   warpgroup 0  softmax for Q0 (thread t owns TMEM lane t = query row t), epilogue of Q0
+//   warpgroup 1  softmax for Q1, epilogue of Q1
+//   warpgroup 2  warp 8: TMA producer (Q0/Q1 per work tile, then K_j, V_j into a ring of
+//                shared-memory slots); warp 9: MMA issuer (one thread) and TMEM owner;
+//                warps 10-11 idle.
+// With 12 warps, at most 3 share an SM sub-partition, so each thread gets up to 168
+// registers: enough for a softmax thread to hold its whole 128-score row.
 // The two query tiles ping-pong: while one warpgroup exponentiates S_0, the tensor core
-// computes P_1 V and S_1 for the other, so the MMA pipe and the exponential units
-// overlap.
+// computes P_1 V and S_1 for the other.  Across work tiles the pipeline does not drain:
+// the K/V ring keeps streaming, and a warpgroup's epilogue of tile w overlaps the other
+// warpgroup's last key tile and the first MMAs of tile w+1.
 //
 // Online-softmax details:
 //   * Scores are handled in log2 units, u = s * scale * log2(e), so P = exp2(u - m) is one
@@ -53,11 +63,10 @@ namespace tc {
 
 constexpr int BM = 128;                       // query rows per Q tile (= TMEM lanes)
 constexpr int BN = 128;                       // keys per K/V tile
-constexpr int NQ = 2;                         // Q tiles per CTA
-constexpr int kSoftmaxWarps = 4 * NQ;
-constexpr int kLoadWarp = kSoftmaxWarps;      // warp 8
-constexpr int kMmaWarp = kSoftmaxWarps + 1;   // warp 9
-constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+constexpr int NQ = 2;                         // Q tiles per work tile
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 384;                 // 3 warpgroups
 constexpr int kTmemCols = 512;                // S0 | S1 | O0 | O1, 128 columns each
 constexpr float kRescaleLog2 = 8.0f;          // lazy-rescale threshold (log2 units)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -73,13 +82,14 @@ struct Layout {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + NQ * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-  // barriers: q_full | kv_full[S] | kv_empty[S] | s_full[NQ] | p_full[NQ] | o_full[NQ] | drain
-  static constexpr int kBarQFull = 0;
-  static constexpr int kBarKvFull = 1;
+  // barriers
+  static constexpr int kBarQFull = 0;                     // [NQ]
+  static constexpr int kBarQEmpty = kBarQFull + NQ;       // [NQ]
+  static constexpr int kBarKvFull = kBarQEmpty + NQ;      // [kStages]
   static constexpr int kBarKvEmpty = kBarKvFull + kStages;
-  static constexpr int kBarSFull = kBarKvEmpty + kStages;
-  static constexpr int kBarPFull = kBarSFull + NQ;
-  static constexpr int kBarOFull = kBarPFull + NQ;
+  static constexpr int kBarSFull = kBarKvEmpty + kStages; // [NQ]
+  static constexpr int kBarPFull = kBarSFull + NQ;        // [NQ]
+  static constexpr int kBarOFull = kBarPFull + NQ;        // [NQ]
   static constexpr int kBarDrain = kBarOFull + NQ;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // u32 tmem base, int abort flag
@@ -96,7 +106,10 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   int Hq, Hkv, N;
-  int n_qpairs;        // ceil(N / (NQ * BM)) query-tile pairs per head
+  int n_bh;            // B * Hq
+  int n_qp;            // ceil(N / 256): query-tile pairs per head
+  int units_per_head;  // ceil(n_qp / 2)
+  int n_units;         // n_bh * units_per_head
   int causal;
   int window;          // <= 0: off
   float scale_log2;    // scale * log2(e)
@@ -147,6 +160,47 @@ __device__ __forceinline__ TileRange tile_range(int r0, int N, int nkv, int caus
 
 __device__ __forceinline__ bool participates(const TileRange& t, int j) { return t.active && j >= t.lo && j < t.hi; }
 
+// One work tile: (batch*head, query-tile pair) and the key tiles it streams.
+struct WorkTile {
+  int bh, kvh;
+  TileRange tr0, tr1;
+  int lo, hi;  // union key-tile range
+  __device__ const TileRange& tr(int i) const { return i == 0 ? tr0 : tr1; }
+};
+
+__device__ __forceinline__ WorkTile make_work_tile(const Params& p, int bh, int qp) {
+  WorkTile w;
+  w.bh = bh;
+  const int b = bh / p.Hq;
+  const int hq = bh - b * p.Hq;
+  w.kvh = b * p.Hkv + hq / (p.Hq / p.Hkv);
+  const int nkv = (p.N + BN - 1) / BN;
+  w.tr0 = tile_range(qp * NQ * BM, p.N, nkv, p.causal, p.window);
+  w.tr1 = tile_range(qp * NQ * BM + BM, p.N, nkv, p.causal, p.window);
+  w.lo = w.tr0.lo;
+  w.hi = w.tr0.hi;
+  if (w.tr1.active) {
+    w.lo = min(w.lo, w.tr1.lo);
+    w.hi = max(w.hi, w.tr1.hi);
+  }
+  return w;
+}
+
+// The static schedule: CTA c takes units c, c + G, ...; unit u is head u / U, pair index
+// p = u % U, and covers q-pairs n_qp-1-p (longer under causal) and p (when distinct).
+// Every role walks the same sequence; the callback returns false to stop (abort).
+template <typename F>
+__device__ __forceinline__ void for_each_tile(const Params& p, F&& f) {
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    const int bh = u / p.units_per_head;
+    const int pi = u - bh * p.units_per_head;
+    const int qa = p.n_qp - 1 - pi;
+    for (int half = 0; half < (pi != qa ? 2 : 1); ++half) {  // one call site: f inlines once
+      if (!f(make_work_tile(p, bh, half == 0 ? qa : pi))) return;
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -160,39 +214,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- work tile: (batch*head, query-tile pair), longest rows first within a head
-  const int tile = blockIdx.x;
-  const int bh = tile / p.n_qpairs;
-  const int qp = p.n_qpairs - 1 - (tile - bh * p.n_qpairs);
-  const int b = bh / p.Hq;
-  const int hq = bh - b * p.Hq;
-  const int kvh = b * p.Hkv + hq / (p.Hq / p.Hkv);
-  const int N = p.N;
-  const int nkv = (N + BN - 1) / BN;
-  TileRange tr[NQ];
-#pragma unroll
-  for (int i = 0; i < NQ; ++i) tr[i] = tile_range(qp * NQ * BM + i * BM, N, nkv, p.causal, p.window);
-  int lo = tr[0].lo, hi = tr[0].hi;
-#pragma unroll
-  for (int i = 1; i < NQ; ++i)
-    if (tr[i].active) {
-      lo = min(lo, tr[i].lo);
-      hi = max(hi, tr[i].hi);
-    }
-  const int T = hi - lo;  // key tiles this CTA streams
+  const int wg = warp >> 2;
 
   // ---- set-up: barriers, abort flag, TMEM
   if (threadIdx.x == 0) {
-    mbar_init(&bars[L::kBarQFull], 1);
-    for (int s = 0; s < L::kStages; ++s) {
-      mbar_init(&bars[L::kBarKvFull + s], 1);
-      mbar_init(&bars[L::kBarKvEmpty + s], 1);
-    }
     for (int i = 0; i < NQ; ++i) {
+      mbar_init(&bars[L::kBarQFull + i], 1);
+      mbar_init(&bars[L::kBarQEmpty + i], 1);
       mbar_init(&bars[L::kBarSFull + i], 1);
       mbar_init(&bars[L::kBarPFull + i], 128);
       mbar_init(&bars[L::kBarOFull + i], 1);
+    }
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&bars[L::kBarKvFull + s], 1);
+      mbar_init(&bars[L::kBarKvEmpty + s], 1);
     }
     mbar_init(&bars[L::kBarDrain], 1);
     *abort_flag = 0;
@@ -207,273 +242,271 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
   const WaitCtl ctl{abort_flag, p.timeout_ns};
-  const WaitCtl drain_ctl{abort_flag, 50ull * 1000 * 1000};
+  constexpr unsigned long long kDrainNs = 50ull * 1000 * 1000;
 
-  if (warp == kLoadWarp) {
-    // =========================== TMA producer ===========================
-    if (lane == 0) {
+  if (wg == 2) {
+    if (warp == kLoadWarp && lane == 0) {
+      // =========================== TMA producer ===========================
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       uint8_t* sQ = smem + L::kQOff;
-      uint32_t qbytes = 0;
-#pragma unroll
-      for (int i = 0; i < NQ; ++i) qbytes += tr[i].active ? L::kTileBytes : 0;
-      mbar_arrive_expect_tx(&bars[L::kBarQFull], qbytes);
-#pragma unroll
-      for (int i = 0; i < NQ; ++i)
-        if (tr[i].active)
-          for (int h = 0; h < L::kHalves; ++h)
-            tma_load_3d(sQ + i * L::kTileBytes + h * L::kHalfBytes, &tmQ, &bars[L::kBarQFull], h * 64, tr[i].r0,
-                        bh);
+      uint32_t q_cnt[NQ] = {0, 0};
       int issued = 0;  // loads issued into the ring (K and V alternate)
-      for (int n = 0; n < T && !*abort_flag; ++n) {
-        const int j = lo + n;
-        for (int which = 0; which < 2; ++which) {
-          const int s = issued % L::kStages;
-          const uint32_t fill = issued / L::kStages;
-          if (!mbar_wait(&bars[L::kBarKvEmpty + s], (fill & 1u) ^ 1u, ctl)) break;
-          uint8_t* dst = smem + L::kRingOff + s * L::kTileBytes;
-          mbar_arrive_expect_tx(&bars[L::kBarKvFull + s], L::kTileBytes);
+      for_each_tile(p, [&](const WorkTile& w) {
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+          const TileRange& t = w.tr(i);
+          if (!t.active) continue;
+          if (!mbar_wait(&bars[L::kBarQEmpty + i], (q_cnt[i] & 1u) ^ 1u, ctl)) return false;
+          mbar_arrive_expect_tx(&bars[L::kBarQFull + i], L::kTileBytes);
           for (int h = 0; h < L::kHalves; ++h)
-            tma_load_3d(dst + h * L::kHalfBytes, which ? &tmV : &tmK, &bars[L::kBarKvFull + s], h * 64, j * BN,
-                        kvh);
-          ++issued;
+            tma_load_3d(sQ + i * L::kTileBytes + h * L::kHalfBytes, &tmQ, &bars[L::kBarQFull + i], h * 64, t.r0,
+                        w.bh);
+          ++q_cnt[i];
         }
-      }
+        for (int j = w.lo; j < w.hi; ++j) {
+          for (int which = 0; which < 2; ++which) {
+            const int s = issued % L::kStages;
+            const uint32_t fill = issued / L::kStages;
+            if (!mbar_wait(&bars[L::kBarKvEmpty + s], (fill & 1u) ^ 1u, ctl)) return false;
+            uint8_t* dst = smem + L::kRingOff + s * L::kTileBytes;
+            mbar_arrive_expect_tx(&bars[L::kBarKvFull + s], L::kTileBytes);
+            for (int h = 0; h < L::kHalves; ++h)
+              tma_load_3d(dst + h * L::kHalfBytes, which ? &tmV : &tmK, &bars[L::kBarKvFull + s], h * 64, j * BN,
+                          w.kvh);
+            ++issued;
+          }
+        }
+        return true;
+      });
       if (*abort_flag) {
         // let the copies already in flight land before the CTA's shared memory goes away
         int no_abort = 0;
-        const WaitCtl c{&no_abort, drain_ctl.limit_ns};
-        mbar_wait(&bars[L::kBarQFull], 0, c);
+        const WaitCtl c{&no_abort, kDrainNs};
+        for (int i = 0; i < NQ; ++i)
+          if (q_cnt[i] > 0) mbar_wait(&bars[L::kBarQFull + i], (q_cnt[i] - 1) & 1u, c);
         for (int k = issued - 1; k >= 0 && k >= issued - L::kStages; --k)
           mbar_wait(&bars[L::kBarKvFull + (k % L::kStages)], (k / L::kStages) & 1u, c);
       }
-    }
-  } else if (warp == kMmaWarp) {
-    // =========================== MMA issuer ===========================
-    if (lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
+      // =========================== MMA issuer ===========================
       constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);  // Q (K-major) x K (K-major)
       constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, D, 0, 1);  // P (TMEM) x V (MN-major)
       const uint32_t sQ = smem_addr(smem + L::kQOff);
       const uint32_t sRing = smem_addr(smem + L::kRingOff);
-      bool ok = mbar_wait(&bars[L::kBarQFull], 0, ctl);
-      tc_fence_after();
-      uint32_t p_phase[NQ] = {};
-      uint32_t o_acc[NQ] = {};
+      uint32_t q_cnt[NQ] = {0, 0};
+      uint32_t p_phase[NQ] = {0, 0};
+      int used = 0;  // ring loads consumed before the current work tile
 
-      auto issue_s = [&](int i, uint32_t k_tile) {
-        const uint32_t q_tile = sQ + i * L::kTileBytes;
+      for_each_tile(p, [&](const WorkTile& w) {
+        uint32_t o_acc[NQ] = {0, 0};
+        const int T = w.hi - w.lo;
+        for (int n = 0; n <= T; ++n) {
+          const int j = w.lo + n;
+          const int kidx = used + 2 * n;
+          const int vidx = kidx - 1;
+          const int kslot = kidx % L::kStages;
+          const int vslot = vidx % L::kStages;
+          if (n < T && !mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
+          if (n > 0 && !mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
-          mma_ss(tmem + L::col_s(i), smem_desc_sw128(q_tile + off, 16, 1024), smem_desc_sw128(k_tile + off, 16, 1024),
-                 kIdescS, kk > 0);
-        }
-        mma_commit(&bars[L::kBarSFull + i]);
-      };
-      auto issue_pv = [&](int i, uint32_t v_tile) {
+          for (int i = 0; i < NQ; ++i) {
+            const TileRange& t = w.tr(i);
+            if (n > 0 && participates(t, j - 1)) {
+              if (!mbar_wait(&bars[L::kBarPFull + i], p_phase[i], ctl)) return false;
+              p_phase[i] ^= 1u;
+              tc_fence_after();
+              // O_i (+)= P_i V: A = 16 keys of P = 8 TMEM columns per step; B = 16 key rows
+              // of V (128 B each); the two 64-column slabs of V are kHalfBytes apart
+              const uint32_t v_tile = sRing + vslot * L::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // A: 16 keys of P = 8 TMEM columns; B: 16 key rows of V (128 B each), the two
-          // 64-column slabs of V are L::kHalfBytes apart (leading byte offset)
-          mma_ts(tmem + L::col_o(i), tmem + L::col_s(i) + kk * 8,
-                 smem_desc_sw128(v_tile + kk * 16 * 128, L::kHalfBytes, 1024), kIdescPV, (kk > 0) || o_acc[i]);
-        }
-        o_acc[i] = 1;
-      };
-
-      for (int n = 0; ok && n <= T; ++n) {
-        const int j = lo + n;
-        const int kslot = (2 * n) % L::kStages;
-        const int vslot = (2 * n - 1) % L::kStages;
-        if (n < T) {
-          ok = mbar_wait(&bars[L::kBarKvFull + kslot], ((2 * n) / L::kStages) & 1u, ctl);
-          if (!ok) break;
-        }
-        if (n > 0) {
-          ok = mbar_wait(&bars[L::kBarKvFull + vslot], ((2 * n - 1) / L::kStages) & 1u, ctl);
-          if (!ok) break;
-        }
-        tc_fence_after();
+              for (int kk = 0; kk < BN / 16; ++kk)
+                mma_ts(tmem + L::col_o(i), tmem + L::col_s(i) + kk * 8,
+                       smem_desc_sw128(v_tile + kk * 16 * 128, L::kHalfBytes, 1024), kIdescPV, (kk > 0) || o_acc[i]);
+              o_acc[i] = 1;
+              if (!participates(t, j)) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
+            }
+            if (n < T && participates(t, j)) {
+              if (j == t.lo) {  // first use of this work tile's Q_i
+                if (!mbar_wait(&bars[L::kBarQFull + i], q_cnt[i] & 1u, ctl)) return false;
+                ++q_cnt[i];
+                tc_fence_after();
+              }
+              const uint32_t q_tile = sQ + i * L::kTileBytes;
+              const uint32_t k_tile = sRing + kslot * L::kTileBytes;
 #pragma unroll
-        for (int i = 0; i < NQ; ++i) {
-          if (n > 0 && participates(tr[i], j - 1)) {
-            ok = mbar_wait(&bars[L::kBarPFull + i], p_phase[i], ctl);
-            if (!ok) break;
-            p_phase[i] ^= 1u;
-            tc_fence_after();
-            issue_pv(i, sRing + vslot * L::kTileBytes);
-            if (!participates(tr[i], j)) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
+                mma_ss(tmem + L::col_s(i), smem_desc_sw128(q_tile + off, 16, 1024),
+                       smem_desc_sw128(k_tile + off, 16, 1024), kIdescS, kk > 0);
+              }
+              mma_commit(&bars[L::kBarSFull + i]);
+              if (j == t.hi - 1) mma_commit(&bars[L::kBarQEmpty + i]);  // Q_i no longer read
+            }
           }
-          if (n < T && participates(tr[i], j)) issue_s(i, sRing + kslot * L::kTileBytes);
+          if (n < T) mma_commit(&bars[L::kBarKvEmpty + kslot]);
+          if (n > 0) mma_commit(&bars[L::kBarKvEmpty + vslot]);
         }
-        if (!ok) break;
-        if (n < T) mma_commit(&bars[L::kBarKvEmpty + kslot]);
-        if (n > 0) mma_commit(&bars[L::kBarKvEmpty + vslot]);
-      }
+        used += 2 * T;
+        return true;
+      });
       // make sure nothing this thread issued is still running before TMEM is released
       mma_commit(&bars[L::kBarDrain]);
       int no_abort = 0;
-      mbar_wait(&bars[L::kBarDrain], 0, WaitCtl{&no_abort, drain_ctl.limit_ns});
+      mbar_wait(&bars[L::kBarDrain], 0, WaitCtl{&no_abort, kDrainNs});
     }
   } else {
     // =========================== softmax warpgroups ===========================
-    const int i = warp >> 2;       // which Q tile
-    const int wq = warp & 3;       // TMEM lane quarter of this warp
+    const int i = wg;               // which Q tile
+    const int wq = warp & 3;        // TMEM lane quarter of this warp
     const int trow = wq * 32 + lane;
-    const TileRange t = (i == 0) ? tr[0] : tr[1];
-    const int row = t.r0 + trow;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t colS = L::col_s(i);
     const uint32_t colO = L::col_o(i);
+    uint32_t s_phase = 0, o_phase = 0;
 
-    float m = -CUDART_INF_F;  // running reference maximum (log2 units)
-    float l = 0.f;            // running sum of P (fp32) relative to m
-    float lr = 0.f;           // running sum of the bf16-rounded P relative to m
-    uint32_t s_phase = 0;
-    bool o_valid = false;
-    bool ok = true;
+    for_each_tile(p, [&](const WorkTile& w) {
+      const TileRange& t = w.tr(i);
+      if (!t.active) return true;
+      const int row = t.r0 + trow;
+      float m = -CUDART_INF_F;  // running reference maximum (log2 units)
+      float l = 0.f;            // running sum of P (fp32) relative to m
+      float lr = 0.f;           // running sum of the bf16-rounded P relative to m
+      bool o_valid = false;
 
-    for (int n = 0; n < T && ok; ++n) {
-      const int j = lo + n;
-      if (!participates(t, j)) continue;
-      // tcgen05.ld/st are warp-collective: the whole warp leaves together or not at all
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[L::kBarSFull + i], s_phase, ctl));
-      if (!ok) break;
-      s_phase ^= 1u;
-      tc_fence_after();
-
-      float s[BN];
-      {
-        uint32_t r[32];
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          tmem_ld32_wait(lane_base + colS + c * 32, r);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(r[x]);
-        }
-      }
-
-      const int k0 = j * BN;
-      const bool need_mask = (k0 + BN > N) || (p.causal && k0 + BN - 1 > t.r0) ||
-                             (p.window > 0 && t.r1 - k0 >= p.window);
-      if (need_mask) {
-#pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const int key = k0 + c;
-          bool valid = key < N;
-          if (p.causal && key > row) valid = false;
-          if (p.window > 0 && row - key >= p.window) valid = false;
-          if (!valid) s[c] = -CUDART_INF_F;
-        }
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-      float m_tile;
-      if (p.use_softcap)
-        m_tile = (mx == -CUDART_INF_F) ? -CUDART_INF_F : p.cap_outer * tanh_cap(mx * p.cap_inner);
-      else
-        m_tile = mx * p.scale_log2;
-      const float m_new = fmaxf(m, m_tile);
-
-      if (!o_valid) {
-        m = m_new;  // nothing accumulated yet: adopt the maximum as is
-      } else {
-        const bool need = m_new > m + kRescaleLog2;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
-          if (need) {
-            l *= alpha;
-            lr *= alpha;
-            m = m_new;
-          }
-          uint32_t r[32];
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            tmem_ld32_wait(lane_base + colO + c * 32, r);
-#pragma unroll
-            for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-            tmem_st32(lane_base + colO + c * 32, r);
-          }
-        }
-      }
-      const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
-
-      // P = exp2(u - m), 32 keys at a time: 16 packed bf16 pairs per chunk go straight to
-      // TMEM over the first 64 columns of S_i (two bf16 per 32-bit column).  Two sums are
-      // kept: l (fp32 P) for the log-sum-exp, and lr (the bf16-rounded P that the tensor
-      // core multiplies with V) to normalise O, so O is a weighted mean of V with exactly
-      // the weights the MMA used.
-      float lsum0 = 0.f, lsum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
-#pragma unroll
-      for (int cb = 0; cb < BN / 32; ++cb) {
-        uint32_t packed[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const float a = s[cb * 32 + 2 * x];
-          const float bb = s[cb * 32 + 2 * x + 1];
-          float e0, e1;
-          if (p.use_softcap) {
-            e0 = ex2_approx(fmaf(tanh_cap(a * p.cap_inner), p.cap_outer, -m_use));
-            e1 = ex2_approx(fmaf(tanh_cap(bb * p.cap_inner), p.cap_outer, -m_use));
-            e0 = (a == -CUDART_INF_F) ? 0.f : e0;
-            e1 = (bb == -CUDART_INF_F) ? 0.f : e1;
-          } else {
-            e0 = ex2_approx(fmaf(a, p.scale_log2, -m_use));
-            e1 = ex2_approx(fmaf(bb, p.scale_log2, -m_use));
-          }
-          lsum0 += e0;
-          lsum1 += e1;
-          const uint32_t pk = pack_bf16x2(e0, e1);
-          rsum0 += __uint_as_float(pk << 16);
-          rsum1 += __uint_as_float(pk & 0xFFFF0000u);
-          packed[x] = pk;
-        }
-        tmem_st16(lane_base + colS + cb * 16, packed);
-      }
-      l += lsum0 + lsum1;
-      lr += rsum0 + rsum1;
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars[L::kBarPFull + i]);
-      o_valid = true;
-    }
-
-    // ---- epilogue: O / l -> bf16, LSE = (m + log2 l) ln 2
-    if (ok && t.active) {
-      if (o_valid) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars[L::kBarOFull + i], 0, ctl));
+      for (int j = t.lo; j < t.hi; ++j) {
+        // tcgen05.ld/st are warp-collective: the whole warp leaves together or not at all
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarSFull + i], s_phase, ctl))) return false;
+        s_phase ^= 1u;
         tc_fence_after();
-      }
-      if (ok) {
-        const float inv = lr > 0.f ? 1.0f / lr : 0.f;
-        __nv_bfloat16* orow = p.o + (static_cast<int64_t>(bh) * N + row) * D;
-        uint32_t r[32];
+
+        float s[BN];
+        {
+          uint32_t r[BN];
+          tmem_ld128_wait(lane_base + colS, r);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          if (o_valid) {
-            tmem_ld32_wait(lane_base + colO + c * 32, r);
-          } else {
+          for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
+        }
+
+        const int k0 = j * BN;
+        const bool need_mask = (k0 + BN > p.N) || (p.causal && k0 + BN - 1 > t.r0) ||
+                               (p.window > 0 && t.r1 - k0 >= p.window);
+        if (need_mask) {
 #pragma unroll
-            for (int x = 0; x < 32; ++x) r[x] = 0u;
-          }
-          if (row < N) {
-            uint4 w[4];
-            uint32_t* wp = reinterpret_cast<uint32_t*>(w);
-#pragma unroll
-            for (int x = 0; x < 16; ++x)
-              wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * inv, __uint_as_float(r[2 * x + 1]) * inv);
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) dst[x] = w[x];
+          for (int c = 0; c < BN; ++c) {
+            const int key = k0 + c;
+            bool valid = key < p.N;
+            if (p.causal && key > row) valid = false;
+            if (p.window > 0 && row - key >= p.window) valid = false;
+            if (!valid) s[c] = -CUDART_INF_F;
           }
         }
-        if (p.lse != nullptr && row < N)
-          p.lse[static_cast<int64_t>(bh) * N + row] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < BN; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        float m_tile;
+        if (p.use_softcap)
+          m_tile = (mx == -CUDART_INF_F) ? -CUDART_INF_F : p.cap_outer * tanh_cap(mx * p.cap_inner);
+        else
+          m_tile = mx * p.scale_log2;
+        const float m_new = fmaxf(m, m_tile);
+
+        if (!o_valid) {
+          m = m_new;  // nothing accumulated yet: adopt the maximum as is
+        } else {
+          const bool need = m_new > m + kRescaleLog2;
+          if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
+            if (need) {
+              l *= alpha;
+              lr *= alpha;
+              m = m_new;
+            }
+            uint32_t r[32];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              tmem_ld32_wait(lane_base + colO + c * 32, r);
+#pragma unroll
+              for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+              tmem_st32(lane_base + colO + c * 32, r);
+            }
+          }
+        }
+        const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
+
+        // P = exp2(u - m), 32 keys at a time: 16 packed bf16 pairs per chunk go straight
+        // to TMEM over the first 64 columns of S_i (two bf16 per 32-bit column).  Two sums
+        // are kept: l (fp32 P) for the log-sum-exp, and lr (the bf16-rounded P that the
+        // tensor core multiplies with V) to normalise O, so O is a weighted mean of V with
+        // exactly the weights the MMA used.
+        float lsum0 = 0.f, lsum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
+#pragma unroll
+        for (int cb = 0; cb < BN / 32; ++cb) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const float a = s[cb * 32 + 2 * x];
+            const float bb = s[cb * 32 + 2 * x + 1];
+            float e0, e1;
+            if (p.use_softcap) {
+              e0 = ex2_approx(fmaf(tanh_cap(a * p.cap_inner), p.cap_outer, -m_use));
+              e1 = ex2_approx(fmaf(tanh_cap(bb * p.cap_inner), p.cap_outer, -m_use));
+              e0 = (a == -CUDART_INF_F) ? 0.f : e0;
+              e1 = (bb == -CUDART_INF_F) ? 0.f : e1;
+            } else {
+              e0 = ex2_approx(fmaf(a, p.scale_log2, -m_use));
+              e1 = ex2_approx(fmaf(bb, p.scale_log2, -m_use));
+            }
+            lsum0 += e0;
+            lsum1 += e1;
+            const uint32_t pk = pack_bf16x2(e0, e1);
+            rsum0 += __uint_as_float(pk << 16);
+            rsum1 += __uint_as_float(pk & 0xFFFF0000u);
+            packed[x] = pk;
+          }
+          tmem_st16(lane_base + colS + cb * 16, packed);
+        }
+        l += lsum0 + lsum1;
+        lr += rsum0 + rsum1;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars[L::kBarPFull + i]);
+        o_valid = true;
       }
-    }
+
+      // ---- epilogue: O / lr -> bf16, LSE = (m + log2 l) ln 2
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarOFull + i], o_phase, ctl))) return false;
+      o_phase ^= 1u;
+      tc_fence_after();
+      const float inv = lr > 0.f ? 1.0f / lr : 0.f;
+      __nv_bfloat16* orow = p.o + (static_cast<int64_t>(w.bh) * p.N + row) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32_wait(lane_base + colO + c * 32, r);
+        if (row < p.N) {
+          uint4 v4[4];
+          uint32_t* wp = reinterpret_cast<uint32_t*>(v4);
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * inv, __uint_as_float(r[2 * x + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) dst[x] = v4[x];
+        }
+      }
+      if (p.lse != nullptr && row < p.N)
+        p.lse[static_cast<int64_t>(w.bh) * p.N + row] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+      return true;
+    });
   }
 
   // ---- teardown
