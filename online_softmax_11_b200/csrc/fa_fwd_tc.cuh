@@ -138,6 +138,100 @@ __device__ __forceinline__ float tanh_cap(float x) {
   return copysignf(t, x);
 }
 
+// 2^x for a pair of floats on the FMA pipe instead of the exponential unit.  x is split
+// as n + f with n = round(x) (the 1.5 * 2^23 shifter: after x + M the low mantissa bits
+// of the sum hold n), 2^f on [-1/2, 1/2] is a cubic, and n is added to the exponent
+// field.  The cubic's coefficients were fitted for minimum relative error on
+// [-1/2, 1/2] (Lawson's iteratively reweighted least squares): max relative error
+// 7.5e-5, below the 2^-9 of the bf16 rounding that P goes through next.  x is clamped at
+// -125 so the exponent cannot underflow; callers use this only on tiles with no masked
+// key (x > -inf), where 2^-125 is far below anything that can matter.
+__device__ __forceinline__ float2 exp2_fma_pair(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 shifter = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+  const float2 r = __fadd2_rn(x, shifter);
+  const float2 n = __fadd2_rn(r, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);  // x - n, exact
+  float2 q = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.2426111400f, 0.2426111400f));
+  q = __ffma2_rn(q, f, make_float2(0.6932609677f, 0.6932609677f));
+  q = __ffma2_rn(q, f, make_float2(0.9999280572f, 0.9999280572f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(r.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(r.y) << 23)));
+}
+
+__device__ __forceinline__ float2 ex2_pair(float2 x) { return make_float2(ex2_approx(x.x), ex2_approx(x.y)); }
+
+// tanh for a pair known to satisfy |x| < 0.3 (Taylor terms through x^11), or |x| < 0.12
+// when kShort (terms through x^7; the next term is below 1e-10 there).
+template <bool kShort>
+__device__ __forceinline__ float2 tanh_small_pair(float2 x) {
+  const float2 x2 = __fmul2_rn(x, x);
+  float2 p;
+  if (kShort) {
+    p = __ffma2_rn(make_float2(-17.0f / 315.0f, -17.0f / 315.0f), x2, make_float2(2.0f / 15.0f, 2.0f / 15.0f));
+  } else {
+    p = __ffma2_rn(make_float2(-1382.0f / 155925.0f, -1382.0f / 155925.0f), x2,
+                   make_float2(62.0f / 2835.0f, 62.0f / 2835.0f));
+    p = __ffma2_rn(p, x2, make_float2(-17.0f / 315.0f, -17.0f / 315.0f));
+    p = __ffma2_rn(p, x2, make_float2(2.0f / 15.0f, 2.0f / 15.0f));
+  }
+  p = __ffma2_rn(p, x2, make_float2(-1.0f / 3.0f, -1.0f / 3.0f));
+  p = __fmul2_rn(p, x2);
+  return __ffma2_rn(p, x, x);
+}
+
+// How P is produced from the scores of one tile (chosen per tile, warp-uniformly).
+enum class PMode {
+  kPlainMixed,   // no soft-cap, no masked key: 3 of 4 pairs on ex2, 1 of 4 on the FMA pipe
+  kPlainMufu,    // no soft-cap, masked keys present (-inf -> exactly 0): all pairs on ex2
+  kCapShort,     // soft-cap, every |s * scale / cap| < 0.12
+  kCapLong,      // soft-cap, every |s * scale / cap| < 0.3
+  kCapGeneral,   // soft-cap, anything else (including masked keys)
+};
+
+// P = exp2(u - m) for the 128 scores of this thread's row, written to TMEM as bf16
+// pairs over the first 64 columns of the S tile (32 keys = 16 columns per chunk).
+// Returns the fp32 sum of P (for the log-sum-exp) and the sum of the bf16-rounded P
+// that the tensor core multiplies with V (to normalise O).
+template <PMode kMode>
+__device__ __forceinline__ void make_p(const float (&s)[BN], uint32_t taddr_p, float scale_log2, float cap_inner,
+                                       float cap_outer, float m_use, float& l_out, float& lr_out) {
+  const float2 negm = make_float2(-m_use, -m_use);
+  float2 lsum = make_float2(0.f, 0.f), rsum = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int cb = 0; cb < BN / 32; ++cb) {
+    uint32_t packed[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const float2 sv = make_float2(s[cb * 32 + 2 * x], s[cb * 32 + 2 * x + 1]);
+      float2 e;
+      if constexpr (kMode == PMode::kPlainMixed || kMode == PMode::kPlainMufu) {
+        const float2 u = __ffma2_rn(sv, make_float2(scale_log2, scale_log2), negm);
+        if (kMode == PMode::kPlainMixed && (x & 3) == 3)
+          e = exp2_fma_pair(u);
+        else
+          e = ex2_pair(u);
+      } else if constexpr (kMode == PMode::kCapShort || kMode == PMode::kCapLong) {
+        const float2 t = tanh_small_pair<kMode == PMode::kCapShort>(__fmul2_rn(sv, make_float2(cap_inner, cap_inner)));
+        e = ex2_pair(__ffma2_rn(t, make_float2(cap_outer, cap_outer), negm));
+      } else {
+        e.x = ex2_approx(fmaf(tanh_cap(sv.x * cap_inner), cap_outer, -m_use));
+        e.y = ex2_approx(fmaf(tanh_cap(sv.y * cap_inner), cap_outer, -m_use));
+        e.x = (sv.x == -CUDART_INF_F) ? 0.f : e.x;
+        e.y = (sv.y == -CUDART_INF_F) ? 0.f : e.y;
+      }
+      lsum = __fadd2_rn(lsum, e);
+      const uint32_t pk = pack_bf16x2(e.x, e.y);
+      rsum = __fadd2_rn(rsum, make_float2(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
+      packed[x] = pk;
+    }
+    tmem_st16(taddr_p + cb * 16, packed);
+  }
+  l_out = lsum.x + lsum.y;
+  lr_out = rsum.x + rsum.y;
+}
+
 // Key-tile range of one query tile: [lo, hi) of 128-key tiles.
 struct TileRange {
   int r0, r1;  // first / last query row (r1 < N)
@@ -299,6 +393,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t p_phase[NQ] = {0, 0};
       int used = 0;  // ring loads consumed before the current work tile
 
+      // Descriptor of the first 16-column K step of each operand tile; later steps add
+      // their byte offset / 16 to the start-address field (no carry: addresses < 256 KB),
+      // inside mma_ss_kloop / mma_ts_kloop8.
+      const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dring = smem_desc_sw128(sRing, 16, 1024);
+      const uint64_t dvring = smem_desc_sw128(sRing, L::kHalfBytes, 1024);
+
       for_each_tile(p, [&](const WorkTile& w) {
         uint32_t o_acc[NQ] = {0, 0};
         const int T = w.hi - w.lo;
@@ -308,9 +409,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int vidx = kidx - 1;
           const int kslot = kidx % L::kStages;
           const int vslot = vidx % L::kStages;
-          if (n < T && !mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
-          if (n > 0 && !mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
-          tc_fence_after();
+          // P_i V_{n-1} needs only V_{n-1}; S_i(n) needs K_n: wait for each just before use
+          if (n > 0) {
+            if (!mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
+            tc_fence_after();
+          }
+          bool k_ready = false;
 #pragma unroll
           for (int i = 0; i < NQ; ++i) {
             const TileRange& t = w.tr(i);
@@ -320,33 +424,34 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_after();
               // O_i (+)= P_i V: A = 16 keys of P = 8 TMEM columns per step; B = 16 key rows
               // of V (128 B each); the two 64-column slabs of V are kHalfBytes apart
-              const uint32_t v_tile = sRing + vslot * L::kTileBytes;
-#pragma unroll
-              for (int kk = 0; kk < BN / 16; ++kk)
-                mma_ts(tmem + L::col_o(i), tmem + L::col_s(i) + kk * 8,
-                       smem_desc_sw128(v_tile + kk * 16 * 128, L::kHalfBytes, 1024), kIdescPV, (kk > 0) || o_acc[i]);
+              mma_ts_kloop8(tmem + L::col_o(i), tmem + L::col_s(i), dvring + ((vslot * L::kTileBytes) >> 4), kIdescPV,
+                            o_acc[i]);
               o_acc[i] = 1;
               if (!participates(t, j)) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
             }
             if (n < T && participates(t, j)) {
+              if (!k_ready) {
+                if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
+                k_ready = true;
+                tc_fence_after();
+              }
               if (j == t.lo) {  // first use of this work tile's Q_i
                 if (!mbar_wait(&bars[L::kBarQFull + i], q_cnt[i] & 1u, ctl)) return false;
                 ++q_cnt[i];
                 tc_fence_after();
               }
-              const uint32_t q_tile = sQ + i * L::kTileBytes;
-              const uint32_t k_tile = sRing + kslot * L::kTileBytes;
-#pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
-                mma_ss(tmem + L::col_s(i), smem_desc_sw128(q_tile + off, 16, 1024),
-                       smem_desc_sw128(k_tile + off, 16, 1024), kIdescS, kk > 0);
-              }
+              mma_ss_kloop<D / 16>(tmem + L::col_s(i), dq0 + ((i * L::kTileBytes) >> 4),
+                                   dring + ((kslot * L::kTileBytes) >> 4), kIdescS);
               mma_commit(&bars[L::kBarSFull + i]);
               if (j == t.hi - 1) mma_commit(&bars[L::kBarQEmpty + i]);  // Q_i no longer read
             }
           }
-          if (n < T) mma_commit(&bars[L::kBarKvEmpty + kslot]);
+          if (n < T) {
+            if (!k_ready) {  // no query tile used K_n here (cannot happen), keep the ring in step
+              if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
+            }
+            mma_commit(&bars[L::kBarKvEmpty + kslot]);
+          }
           if (n > 0) mma_commit(&bars[L::kBarKvEmpty + vslot]);
         }
         used += 2 * T;
@@ -403,15 +508,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!valid) s[c] = -CUDART_INF_F;
           }
         }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        // row maximum (and minimum, for the soft-cap range check): four independent
+        // chains of three-input max
+        float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]);
+        float mx2 = fmax3(s[6], s[7], s[8]), mx3 = fmax3(s[9], s[10], s[11]);
 #pragma unroll
-        for (int c = 4; c < BN; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
+        for (int c = 12; c < BN; c += 8) {
+          mx0 = fmax3(mx0, s[c], s[c + 1]);
+          mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+          mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+          mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
         }
-        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float mx = fmax3(fmaxf(mx0, mx1), mx2, mx3);
+        float mn = 0.f;
+        if (p.use_softcap && !need_mask) {
+          float mn0 = fmin3(s[0], s[1], s[2]), mn1 = fmin3(s[3], s[4], s[5]);
+          float mn2 = fmin3(s[6], s[7], s[8]), mn3 = fmin3(s[9], s[10], s[11]);
+#pragma unroll
+          for (int c = 12; c < BN; c += 8) {
+            mn0 = fmin3(mn0, s[c], s[c + 1]);
+            mn1 = fmin3(mn1, s[c + 2], s[c + 3]);
+            mn2 = fmin3(mn2, s[c + 4], s[c + 5]);
+            mn3 = fmin3(mn3, s[c + 6], s[c + 7]);
+          }
+          mn = fmin3(fminf(mn0, mn1), mn2, mn3);
+        }
         float m_tile;
         if (p.use_softcap)
           m_tile = (mx == -CUDART_INF_F) ? -CUDART_INF_F : p.cap_outer * tanh_cap(mx * p.cap_inner);
@@ -442,40 +563,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
 
-        // P = exp2(u - m), 32 keys at a time: 16 packed bf16 pairs per chunk go straight
-        // to TMEM over the first 64 columns of S_i (two bf16 per 32-bit column).  Two sums
-        // are kept: l (fp32 P) for the log-sum-exp, and lr (the bf16-rounded P that the
-        // tensor core multiplies with V) to normalise O, so O is a weighted mean of V with
-        // exactly the weights the MMA used.
-        float lsum0 = 0.f, lsum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
-#pragma unroll
-        for (int cb = 0; cb < BN / 32; ++cb) {
-          uint32_t packed[16];
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const float a = s[cb * 32 + 2 * x];
-            const float bb = s[cb * 32 + 2 * x + 1];
-            float e0, e1;
-            if (p.use_softcap) {
-              e0 = ex2_approx(fmaf(tanh_cap(a * p.cap_inner), p.cap_outer, -m_use));
-              e1 = ex2_approx(fmaf(tanh_cap(bb * p.cap_inner), p.cap_outer, -m_use));
-              e0 = (a == -CUDART_INF_F) ? 0.f : e0;
-              e1 = (bb == -CUDART_INF_F) ? 0.f : e1;
-            } else {
-              e0 = ex2_approx(fmaf(a, p.scale_log2, -m_use));
-              e1 = ex2_approx(fmaf(bb, p.scale_log2, -m_use));
-            }
-            lsum0 += e0;
-            lsum1 += e1;
-            const uint32_t pk = pack_bf16x2(e0, e1);
-            rsum0 += __uint_as_float(pk << 16);
-            rsum1 += __uint_as_float(pk & 0xFFFF0000u);
-            packed[x] = pk;
-          }
-          tmem_st16(lane_base + colS + cb * 16, packed);
+        float lt, lrt;
+        if (!p.use_softcap) {
+          if (need_mask)
+            make_p<PMode::kPlainMufu>(s, lane_base + colS, p.scale_log2, 0.f, 0.f, m_use, lt, lrt);
+          else
+            make_p<PMode::kPlainMixed>(s, lane_base + colS, p.scale_log2, 0.f, 0.f, m_use, lt, lrt);
+        } else {
+          const float amax = fmaxf(fabsf(mx), fabsf(mn)) * p.cap_inner;  // max |x| of the row
+          const int tier = need_mask ? 2 : (amax < 0.12f ? 0 : (amax < 0.3f ? 1 : 2));
+          const int wtier = __reduce_max_sync(0xffffffffu, tier);
+          if (wtier == 0)
+            make_p<PMode::kCapShort>(s, lane_base + colS, 0.f, p.cap_inner, p.cap_outer, m_use, lt, lrt);
+          else if (wtier == 1)
+            make_p<PMode::kCapLong>(s, lane_base + colS, 0.f, p.cap_inner, p.cap_outer, m_use, lt, lrt);
+          else
+            make_p<PMode::kCapGeneral>(s, lane_base + colS, 0.f, p.cap_inner, p.cap_outer, m_use, lt, lrt);
         }
-        l += lsum0 + lsum1;
-        lr += rsum0 + rsum1;
+        l += lt;
+        lr += lrt;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars[L::kBarPFull + i]);

@@ -143,6 +143,71 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// A whole K loop of one 128 x 128 (or 128 x D) product in one asm block, so the issuing
+// thread spends as few instructions as possible between MMAs (the tensor pipe takes one
+// M=128 N=128 K=16 MMA every 64 cycles; a single issuing thread has to keep up).
+//
+// SS form for S = Q K^T with both operands K-major, 128-byte swizzled, d/64 slabs of
+// 128 rows x 128 B: step kk advances the start address by 32 B inside a slab (+2 in the
+// descriptor's 16-byte units) and by one slab (16 KB, +1024) every 4 steps.
+template <int KSTEPS>
+__device__ __forceinline__ void mma_ss_kloop(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
+  static_assert(KSTEPS == 4 || KSTEPS == 8, "d = 64 or 128");
+  asm volatile(
+      "{\n\t.reg .pred pt, pf;\n\t.reg .b64 a, b;\n\t"
+      "setp.eq.u32 pt, 0, 0;\n\t"
+      "setp.ne.u32 pf, 0, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, pf;\n\t"
+      "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+      "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+      "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+      ".reg .pred p8;\n\t"
+      "setp.eq.u32 p8, %4, 8;\n\t"
+      "@!p8 bra.uni MMA_SS_DONE_%=;\n\t"
+      "add.s64 a, %1, 1024;\n\tadd.s64 b, %2, 1024;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+      "add.s64 a, %1, 1026;\n\tadd.s64 b, %2, 1026;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+      "add.s64 a, %1, 1028;\n\tadd.s64 b, %2, 1028;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+      "add.s64 a, %1, 1030;\n\tadd.s64 b, %2, 1030;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
+      "MMA_SS_DONE_%=:\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "n"(KSTEPS)
+      : "memory");
+}
+
+// TS form for O (+)= P V: A = P in TMEM (16 keys = 8 columns per step), B = V MN-major
+// (16 key rows of 128 B = 2048 B per step, +128 in descriptor units).  `accumulate`
+// applies to the first step only (0 for the first key tile of a query tile).
+__device__ __forceinline__ void mma_ts_kloop8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred pt, p0;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.eq.u32 pt, 0, 0;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+      "add.u32 a, %1, 8;\n\tadd.s64 b, %2, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
+      "add.u32 a, %1, 16;\n\tadd.s64 b, %2, 256;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
+      "add.u32 a, %1, 24;\n\tadd.s64 b, %2, 384;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
+      "add.u32 a, %1, 32;\n\tadd.s64 b, %2, 512;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
+      "add.u32 a, %1, 40;\n\tadd.s64 b, %2, 640;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
+      "add.u32 a, %1, 48;\n\tadd.s64 b, %2, 768;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
+      "add.u32 a, %1, 56;\n\tadd.s64 b, %2, 896;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05 operation this thread issued so far is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -279,6 +344,18 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// three-input maximum (sm_100 PTX form of max.f32)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

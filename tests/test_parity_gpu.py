@@ -128,7 +128,9 @@ BF16_CASES = [
     (1, 2, 2, 700, 128, True, 5, 0.0, 1.0),
     (1, 2, 2, 900, 64, True, 200, 0.0, 1.0),
     (1, 2, 1, 1100, 128, True, 256, 50.0, 1.0),  # window + soft-cap
-    (1, 2, 2, 333, 128, False, 0, 5.0, 1.0),     # tight soft-cap
+    (1, 2, 2, 333, 128, False, 0, 5.0, 1.0),     # tight soft-cap: general tanh path
+    (1, 2, 2, 520, 128, True, 0, 20.0, 1.5),     # |s scale / cap| in (0.12, 0.3): long series
+    (1, 2, 2, 520, 64, False, 0, 50.0, 1.0),     # |s scale / cap| < 0.12: short series
     (1, 2, 2, 600, 128, True, 0, 0.0, 8.0),      # large logits: running max moves a lot
     (1, 2, 2, 600, 64, False, 0, 0.0, 8.0),
 ]
