@@ -186,6 +186,27 @@ def emit(obj):
     print(json.dumps(obj), flush=True)
 
 
+def rank_seeds(w, rank: int):
+    """Seeds of rank `rank`'s own batch: every rank processes an independent batch of the
+    workload (weak scaling, no data exchange)."""
+    return tuple(s + 100 * rank for s in w.seeds())
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Maximum of a per-rank time over all ranks (one all-reduce of one number)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world_size: int, flop_per_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return world_size * flop_per_step * steps / (max_ms / 1e3) / 1e12
+
+
 def reference_arm(args, w):
     """The fp64 CPU oracle as the reference implementation (rank 0 only)."""
     ws, rank, _ = dist_env()
@@ -242,7 +263,7 @@ def gpu_arm(args, w):
     fa.load()
 
     # each rank its own batch: seeds shifted by the rank (weak scaling, no data exchange)
-    seeds = tuple(s + 100 * rank for s in w.seeds())
+    seeds = rank_seeds(w, rank)
     q_h, k_h, v_h = workloads.make_inputs(w, seeds=seeds)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     o = torch.empty_like(q)
@@ -282,13 +303,10 @@ def gpu_arm(args, w):
     if fa.check_status() != 0:
         raise RuntimeError("device status word set during the timed region")
 
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, dev)
     flop_per_step = closed_flops(w)
     per_launch_ms = elapsed_ms / args.steps
-    value = ws * flop_per_step * args.steps / (max_ms / 1e3) / 1e12
+    value = job_tflops(ws, flop_per_step, args.steps, max_ms)
 
     # ---- e2e: pinned host inputs -> device, forward, outputs -> pinned host, per step
     e2e = None
@@ -318,14 +336,12 @@ def gpu_arm(args, w):
             e2e_step()
         ee.record(stream)
         torch.cuda.synchronize(dev)
-        te = torch.tensor([es.elapsed_time(ee)], dtype=torch.float64, device=dev)
-        if ws > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te_ms = max_over_ranks(es.elapsed_time(ee), dev)
         h2d = (q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size())
         d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-        e2e = {"value": ws * flop_per_step * n_e2e / (float(te.item()) / 1e3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_tflops(ws, flop_per_step, n_e2e, te_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "ms_per_step": float(te.item()) / n_e2e}
+               "ms_per_step": te_ms / n_e2e}
         del qp, kp, vp, op, lp, qd, kd, vd
 
     # ---- CPU baseline: the fp64 oracle on a bounded row sample (rank 0, N = 1 only)
