@@ -25,8 +25,8 @@
 //   warpgroup 0  softmax for Q0 (thread t owns TMEM lane t = query row t), epilogue of Q0
 //   warpgroup 1  softmax for Q1, epilogue of Q1
 //   warpgroup 2  warp 8: TMA producer (Q0/Q1 per work tile, then K_j, V_j into a ring of
-//                shared-memory slots); warp 9: MMA issuer (one thread) and TMEM owner;
-//                warps 10-11 idle.
+//                shared-memory slots); warps 9 and 10: one MMA-issuing thread per query
+//                tile (warp 9 also owns the TMEM allocation); warp 11 idle.
 // With 12 warps, at most 3 share an SM sub-partition, so each thread gets up to 168
 // registers: enough for a softmax thread to hold its whole 128-score row.
 // The two query tiles ping-pong: while one warpgroup exponentiates S_0, the tensor core
@@ -91,7 +91,7 @@ struct Layout {
   static constexpr int kBarPFull = kBarSFull + NQ;        // [NQ]
   static constexpr int kBarOFull = kBarPFull + NQ;        // [NQ]
   static constexpr int kBarDrain = kBarOFull + NQ;
-  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kNumBars = kBarDrain + NQ;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // u32 tmem base, int abort flag
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;         // slack for 1024-byte alignment
@@ -183,24 +183,24 @@ __device__ __forceinline__ float2 tanh_small_pair(float2 x) {
 
 // How P is produced from the scores of one tile (chosen per tile, warp-uniformly).
 enum class PMode {
-  kPlainMixed,   // no soft-cap, no masked key: 3 of 4 pairs on ex2, 1 of 4 on the FMA pipe
+  kPlainMixed,   // no soft-cap, no masked key: 7 of 8 pairs on ex2, 1 of 8 on the FMA pipe
   kPlainMufu,    // no soft-cap, masked keys present (-inf -> exactly 0): all pairs on ex2
   kCapShort,     // soft-cap, every |s * scale / cap| < 0.12
   kCapLong,      // soft-cap, every |s * scale / cap| < 0.3
   kCapGeneral,   // soft-cap, anything else (including masked keys)
 };
 
-// P = exp2(u - m) for the 128 scores of this thread's row, written to TMEM as bf16
-// pairs over the first 64 columns of the S tile (32 keys = 16 columns per chunk).
-// Returns the fp32 sum of P (for the log-sum-exp) and the sum of the bf16-rounded P
-// that the tensor core multiplies with V (to normalise O).
+constexpr int kHalf = BN / 2;  // the softmax works on 64-score halves of a row
+
+// P = exp2(u - m) for 64 scores of this thread's row, written to TMEM as bf16 pairs
+// (32 keys = 16 columns per chunk) at taddr_p.  Returns the fp32 sum of these P.
 template <PMode kMode>
-__device__ __forceinline__ void make_p(const float (&s)[BN], uint32_t taddr_p, float scale_log2, float cap_inner,
-                                       float cap_outer, float m_use, float& l_out, float& lr_out) {
+__device__ __forceinline__ float make_p(const float (&s)[kHalf], uint32_t taddr_p, float scale_log2, float cap_inner,
+                                        float cap_outer, float m_use) {
   const float2 negm = make_float2(-m_use, -m_use);
-  float2 lsum = make_float2(0.f, 0.f), rsum = make_float2(0.f, 0.f);
+  float2 lsum0 = make_float2(0.f, 0.f), lsum1 = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int cb = 0; cb < BN / 32; ++cb) {
+  for (int cb = 0; cb < kHalf / 32; ++cb) {
     uint32_t packed[16];
 #pragma unroll
     for (int x = 0; x < 16; ++x) {
@@ -208,7 +208,7 @@ __device__ __forceinline__ void make_p(const float (&s)[BN], uint32_t taddr_p, f
       float2 e;
       if constexpr (kMode == PMode::kPlainMixed || kMode == PMode::kPlainMufu) {
         const float2 u = __ffma2_rn(sv, make_float2(scale_log2, scale_log2), negm);
-        if (kMode == PMode::kPlainMixed && (x & 3) == 3)
+        if (kMode == PMode::kPlainMixed && (x & 7) == 7)
           e = exp2_fma_pair(u);
         else
           e = ex2_pair(u);
@@ -221,15 +221,30 @@ __device__ __forceinline__ void make_p(const float (&s)[BN], uint32_t taddr_p, f
         e.x = (sv.x == -CUDART_INF_F) ? 0.f : e.x;
         e.y = (sv.y == -CUDART_INF_F) ? 0.f : e.y;
       }
-      lsum = __fadd2_rn(lsum, e);
-      const uint32_t pk = pack_bf16x2(e.x, e.y);
-      rsum = __fadd2_rn(rsum, make_float2(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
-      packed[x] = pk;
+      if (x & 1)
+        lsum1 = __fadd2_rn(lsum1, e);
+      else
+        lsum0 = __fadd2_rn(lsum0, e);
+      packed[x] = pack_bf16x2(e.x, e.y);
     }
     tmem_st16(taddr_p + cb * 16, packed);
   }
-  l_out = lsum.x + lsum.y;
-  lr_out = rsum.x + rsum.y;
+  const float2 lsum = __fadd2_rn(lsum0, lsum1);
+  return lsum.x + lsum.y;
+}
+
+// 64 scores of the row (tile columns c0 .. c0+63) from TMEM, masked to the row's valid
+// column range [c_lo, c_hi] when the tile needs a mask (-inf outside).
+__device__ __forceinline__ void load_half(uint32_t taddr, int c0, bool need_mask, int c_lo, int c_hi,
+                                          float (&s)[kHalf]) {
+  uint32_t r[kHalf];
+  tmem_ld64_wait(taddr, r);
+#pragma unroll
+  for (int c = 0; c < kHalf; ++c) s[c] = __uint_as_float(r[c]);
+  if (need_mask) {
+#pragma unroll
+    for (int c = 0; c < kHalf; ++c) s[c] = (c0 + c < c_lo || c0 + c > c_hi) ? -CUDART_INF_F : s[c];
+  }
 }
 
 // Key-tile range of one query tile: [lo, hi) of 128-key tiles.
@@ -321,9 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&bars[L::kBarKvFull + s], 1);
-      mbar_init(&bars[L::kBarKvEmpty + s], 1);
+      mbar_init(&bars[L::kBarKvEmpty + s], NQ);  // released by both MMA issuers
     }
-    mbar_init(&bars[L::kBarDrain], 1);
+    for (int i = 0; i < NQ; ++i) mbar_init(&bars[L::kBarDrain + i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -383,25 +398,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = issued - 1; k >= 0 && k >= issued - L::kStages; --k)
           mbar_wait(&bars[L::kBarKvFull + (k % L::kStages)], (k / L::kStages) & 1u, c);
       }
-    } else if (warp == kMmaWarp && lane == 0) {
-      // =========================== MMA issuer ===========================
+    } else if ((warp == kMmaWarp || warp == kMmaWarp + 1) && lane == 0) {
+      // =========================== MMA issuers ===========================
+      // One issuing thread per query tile (warp 9: Q0, warp 10: Q1).  Each thread's chain
+      // P_i V -> Q_i K^T is ordered by issue order (S_i overwrites the columns P_i was read
+      // from); the two chains are independent, so one thread's waits and commits overlap
+      // the other's MMAs.  Every K/V slot is released by both issuers (count 2): with a
+      // commit after the MMAs that read it, or a plain arrive when its query tile does not
+      // use that key tile (after the fill has landed, so a thread can never arrive ahead
+      // into the slot's next phase).
+      const int i = warp - kMmaWarp;
       constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);  // Q (K-major) x K (K-major)
       constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, D, 0, 1);  // P (TMEM) x V (MN-major)
-      const uint32_t sQ = smem_addr(smem + L::kQOff);
-      const uint32_t sRing = smem_addr(smem + L::kRingOff);
-      uint32_t q_cnt[NQ] = {0, 0};
-      uint32_t p_phase[NQ] = {0, 0};
-      int used = 0;  // ring loads consumed before the current work tile
-
       // Descriptor of the first 16-column K step of each operand tile; later steps add
       // their byte offset / 16 to the start-address field (no carry: addresses < 256 KB),
       // inside mma_ss_kloop / mma_ts_kloop8.
-      const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
-      const uint64_t dring = smem_desc_sw128(sRing, 16, 1024);
-      const uint64_t dvring = smem_desc_sw128(sRing, L::kHalfBytes, 1024);
+      const uint64_t dq = smem_desc_sw128(smem_addr(smem + L::kQOff + i * L::kTileBytes), 16, 1024);
+      const uint64_t dring = smem_desc_sw128(smem_addr(smem + L::kRingOff), 16, 1024);
+      const uint64_t dvring = smem_desc_sw128(smem_addr(smem + L::kRingOff), L::kHalfBytes, 1024);
+      const uint32_t d_s = tmem + L::col_s(i);
+      const uint32_t d_o = tmem + L::col_o(i);
+      uint32_t q_cnt = 0, p_phase = 0;
+      int used = 0;  // ring loads consumed before the current work tile
 
       for_each_tile(p, [&](const WorkTile& w) {
-        uint32_t o_acc[NQ] = {0, 0};
+        const TileRange& t = w.tr(i);
+        uint32_t o_acc = 0;
         const int T = w.hi - w.lo;
         for (int n = 0; n <= T; ++n) {
           const int j = w.lo + n;
@@ -409,58 +431,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int vidx = kidx - 1;
           const int kslot = kidx % L::kStages;
           const int vslot = vidx % L::kStages;
-          // P_i V_{n-1} needs only V_{n-1}; S_i(n) needs K_n: wait for each just before use
+          // TMA -> MMA hand-offs (K, V, Q) need only the mbarrier (both sides are async
+          // proxy on shared memory).  P, written to tensor memory by the softmax warps'
+          // tcgen05.st, also needs tcgen05.fence::after_thread_sync after its barrier.
           if (n > 0) {
-            if (!mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
-            tc_fence_after();
-          }
-          bool k_ready = false;
-#pragma unroll
-          for (int i = 0; i < NQ; ++i) {
-            const TileRange& t = w.tr(i);
-            if (n > 0 && participates(t, j - 1)) {
-              if (!mbar_wait(&bars[L::kBarPFull + i], p_phase[i], ctl)) return false;
-              p_phase[i] ^= 1u;
+            if (participates(t, j - 1)) {
+              if (!mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
+              if (!mbar_wait(&bars[L::kBarPFull + i], p_phase, ctl)) return false;
+              p_phase ^= 1u;
               tc_fence_after();
               // O_i (+)= P_i V: A = 16 keys of P = 8 TMEM columns per step; B = 16 key rows
               // of V (128 B each); the two 64-column slabs of V are kHalfBytes apart
-              mma_ts_kloop8(tmem + L::col_o(i), tmem + L::col_s(i), dvring + ((vslot * L::kTileBytes) >> 4), kIdescPV,
-                            o_acc[i]);
-              o_acc[i] = 1;
+              mma_ts_kloop8(d_o, d_s, dvring + ((vslot * L::kTileBytes) >> 4), kIdescPV, o_acc);
+              o_acc = 1;
               if (!participates(t, j)) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
-            }
-            if (n < T && participates(t, j)) {
-              if (!k_ready) {
-                if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
-                k_ready = true;
-                tc_fence_after();
-              }
-              if (j == t.lo) {  // first use of this work tile's Q_i
-                if (!mbar_wait(&bars[L::kBarQFull + i], q_cnt[i] & 1u, ctl)) return false;
-                ++q_cnt[i];
-                tc_fence_after();
-              }
-              mma_ss_kloop<D / 16>(tmem + L::col_s(i), dq0 + ((i * L::kTileBytes) >> 4),
-                                   dring + ((kslot * L::kTileBytes) >> 4), kIdescS);
-              mma_commit(&bars[L::kBarSFull + i]);
-              if (j == t.hi - 1) mma_commit(&bars[L::kBarQEmpty + i]);  // Q_i no longer read
+              mma_commit(&bars[L::kBarKvEmpty + vslot]);
+            } else {
+              // not used by this query tile: release it, but only once this fill has
+              // landed, so the arrive cannot be counted towards the slot's next fill
+              if (!mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
+              mbar_arrive(&bars[L::kBarKvEmpty + vslot]);
             }
           }
           if (n < T) {
-            if (!k_ready) {  // no query tile used K_n here (cannot happen), keep the ring in step
+            if (participates(t, j)) {
               if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
+              if (j == t.lo) {  // first use of this work tile's Q_i
+                if (!mbar_wait(&bars[L::kBarQFull + i], q_cnt & 1u, ctl)) return false;
+                ++q_cnt;
+              }
+              mma_ss_kloop<D / 16>(d_s, dq, dring + ((kslot * L::kTileBytes) >> 4), kIdescS);
+              mma_commit(&bars[L::kBarSFull + i]);
+              if (j == t.hi - 1) mma_commit(&bars[L::kBarQEmpty + i]);  // Q_i no longer read
+              mma_commit(&bars[L::kBarKvEmpty + kslot]);
+            } else {
+              if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
+              mbar_arrive(&bars[L::kBarKvEmpty + kslot]);
             }
-            mma_commit(&bars[L::kBarKvEmpty + kslot]);
           }
-          if (n > 0) mma_commit(&bars[L::kBarKvEmpty + vslot]);
         }
         used += 2 * T;
         return true;
       });
       // make sure nothing this thread issued is still running before TMEM is released
-      mma_commit(&bars[L::kBarDrain]);
+      mma_commit(&bars[L::kBarDrain + i]);
       int no_abort = 0;
-      mbar_wait(&bars[L::kBarDrain], 0, WaitCtl{&no_abort, kDrainNs});
+      mbar_wait(&bars[L::kBarDrain + i], 0, WaitCtl{&no_abort, kDrainNs});
     }
   } else {
     // =========================== softmax warpgroups ===========================
@@ -478,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = t.r0 + trow;
       float m = -CUDART_INF_F;  // running reference maximum (log2 units)
       float l = 0.f;            // running sum of P (fp32) relative to m
-      float lr = 0.f;           // running sum of the bf16-rounded P relative to m
+      float lr = 0.f;           // normaliser of O (l with each tile maximum's P as rounded)
       bool o_valid = false;
 
       for (int j = t.lo; j < t.hi; ++j) {
@@ -487,52 +503,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         s_phase ^= 1u;
         tc_fence_after();
 
-        float s[BN];
-        {
-          uint32_t r[BN];
-          tmem_ld128_wait(lane_base + colS, r);
-#pragma unroll
-          for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
-        }
-
         const int k0 = j * BN;
         const bool need_mask = (k0 + BN > p.N) || (p.causal && k0 + BN - 1 > t.r0) ||
                                (p.window > 0 && t.r1 - k0 >= p.window);
-        if (need_mask) {
+        // valid keys of this row form one column range [c_lo, c_hi] of the tile: keys
+        // below N, at most the query's own position (causal), and within the window
+        int c_hi = min(BN - 1, p.N - 1 - k0);
+        if (p.causal) c_hi = min(c_hi, row - k0);
+        const int c_lo = p.window > 0 ? max(0, row - p.window + 1 - k0) : 0;
+
+        // Pass 1: row maximum (and minimum, for the soft-cap range check) over the two
+        // 64-score halves (four chains of three-input max), and the maximum of the
+        // columns whose exp2 runs on the FMA pipe in unmasked plain tiles (pairs 7 and 15
+        // of each 32-column chunk), to recompute the tile maximum's P with the very
+        // arithmetic that produced it.
+        float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F, mx2 = -CUDART_INF_F, mx3 = -CUDART_INF_F;
+        float mn0 = CUDART_INF_F, mn1 = CUDART_INF_F;
+        float mx_emu = -CUDART_INF_F;
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const int key = k0 + c;
-            bool valid = key < p.N;
-            if (p.causal && key > row) valid = false;
-            if (p.window > 0 && row - key >= p.window) valid = false;
-            if (!valid) s[c] = -CUDART_INF_F;
+        for (int h = 0; h < 2; ++h) {
+          float s[kHalf];
+          load_half(lane_base + colS + h * kHalf, h * kHalf, need_mask, c_lo, c_hi, s);
+#pragma unroll
+          for (int c = 0; c < kHalf; c += 8) {
+            mx0 = fmax3(mx0, s[c], s[c + 1]);
+            mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+            mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+            mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
           }
-        }
-        // row maximum (and minimum, for the soft-cap range check): four independent
-        // chains of three-input max
-        float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]);
-        float mx2 = fmax3(s[6], s[7], s[8]), mx3 = fmax3(s[9], s[10], s[11]);
+          mx_emu = fmax3(mx_emu, fmax3(s[14], s[15], s[30]), fmax3(s[31], s[46], s[47]));
+          mx_emu = fmax3(mx_emu, s[62], s[63]);
+          if (p.use_softcap) {
 #pragma unroll
-        for (int c = 12; c < BN; c += 8) {
-          mx0 = fmax3(mx0, s[c], s[c + 1]);
-          mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
-          mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
-          mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+            for (int c = 0; c < kHalf; c += 4) {
+              mn0 = fmin3(mn0, s[c], s[c + 1]);
+              mn1 = fmin3(mn1, s[c + 2], s[c + 3]);
+            }
+          }
         }
         const float mx = fmax3(fmaxf(mx0, mx1), mx2, mx3);
-        float mn = 0.f;
-        if (p.use_softcap && !need_mask) {
-          float mn0 = fmin3(s[0], s[1], s[2]), mn1 = fmin3(s[3], s[4], s[5]);
-          float mn2 = fmin3(s[6], s[7], s[8]), mn3 = fmin3(s[9], s[10], s[11]);
-#pragma unroll
-          for (int c = 12; c < BN; c += 8) {
-            mn0 = fmin3(mn0, s[c], s[c + 1]);
-            mn1 = fmin3(mn1, s[c + 2], s[c + 3]);
-            mn2 = fmin3(mn2, s[c + 4], s[c + 5]);
-            mn3 = fmin3(mn3, s[c + 6], s[c + 7]);
-          }
-          mn = fmin3(fminf(mn0, mn1), mn2, mn3);
-        }
+        const float mn = fminf(mn0, mn1);
         float m_tile;
         if (p.use_softcap)
           m_tile = (mx == -CUDART_INF_F) ? -CUDART_INF_F : p.cap_outer * tanh_cap(mx * p.cap_inner);
@@ -563,25 +573,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
 
-        float lt, lrt;
-        if (!p.use_softcap) {
-          if (need_mask)
-            make_p<PMode::kPlainMufu>(s, lane_base + colS, p.scale_log2, 0.f, 0.f, m_use, lt, lrt);
-          else
-            make_p<PMode::kPlainMixed>(s, lane_base + colS, p.scale_log2, 0.f, 0.f, m_use, lt, lrt);
-        } else {
+        // Pass 2: per half, reload the scores, P = exp2(u - m) into TMEM over columns
+        // [32 h, 32 h + 32) of S (already consumed: half 0 was reloaded first).
+        // lt: fp32 sum of this tile's P; pmax: the P of the tile maximum, recomputed with
+        // the same instructions as in make_p (so it is bit-identical to the value packed).
+        float lt = 0.f, pmax;
+        int wtier = 0;
+        if (p.use_softcap) {
           const float amax = fmaxf(fabsf(mx), fabsf(mn)) * p.cap_inner;  // max |x| of the row
           const int tier = need_mask ? 2 : (amax < 0.12f ? 0 : (amax < 0.3f ? 1 : 2));
-          const int wtier = __reduce_max_sync(0xffffffffu, tier);
-          if (wtier == 0)
-            make_p<PMode::kCapShort>(s, lane_base + colS, 0.f, p.cap_inner, p.cap_outer, m_use, lt, lrt);
-          else if (wtier == 1)
-            make_p<PMode::kCapLong>(s, lane_base + colS, 0.f, p.cap_inner, p.cap_outer, m_use, lt, lrt);
-          else
-            make_p<PMode::kCapGeneral>(s, lane_base + colS, 0.f, p.cap_inner, p.cap_outer, m_use, lt, lrt);
+          wtier = __reduce_max_sync(0xffffffffu, tier);
         }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float s[kHalf];
+          load_half(lane_base + colS + h * kHalf, h * kHalf, need_mask, c_lo, c_hi, s);
+          const uint32_t tp = lane_base + colS + h * (kHalf / 2);
+          if (!p.use_softcap) {
+            if (need_mask)
+              lt += make_p<PMode::kPlainMufu>(s, tp, p.scale_log2, 0.f, 0.f, m_use);
+            else
+              lt += make_p<PMode::kPlainMixed>(s, tp, p.scale_log2, 0.f, 0.f, m_use);
+          } else if (wtier == 0) {
+            lt += make_p<PMode::kCapShort>(s, tp, 0.f, p.cap_inner, p.cap_outer, m_use);
+          } else if (wtier == 1) {
+            lt += make_p<PMode::kCapLong>(s, tp, 0.f, p.cap_inner, p.cap_outer, m_use);
+          } else {
+            lt += make_p<PMode::kCapGeneral>(s, tp, 0.f, p.cap_inner, p.cap_outer, m_use);
+          }
+        }
+        if (!p.use_softcap) {
+          const float u = fmaf(mx, p.scale_log2, -m_use);
+          pmax = (!need_mask && mx_emu == mx) ? exp2_fma_pair(make_float2(u, u)).x : ex2_approx(u);
+        } else {
+          const float xm = mx * p.cap_inner;
+          if (wtier == 0)
+            pmax = ex2_approx(fmaf(tanh_small_pair<true>(make_float2(xm, xm)).x, p.cap_outer, -m_use));
+          else if (wtier == 1)
+            pmax = ex2_approx(fmaf(tanh_small_pair<false>(make_float2(xm, xm)).x, p.cap_outer, -m_use));
+          else
+            pmax = ex2_approx(fmaf(tanh_cap(xm), p.cap_outer, -m_use));
+        }
+        if (mx == -CUDART_INF_F) pmax = 0.f;
+        // The normaliser of O is the fp32 sum with the tile maximum's term replaced by its
+        // bf16-rounded value, the weight the tensor core actually multiplied V with.  With
+        // a stale reference the largest P of a row can be up to 256 and is not exact in
+        // bf16; that one term dominates peaked rows, the other roundings average out.
         l += lt;
-        lr += lrt;
+        lr += lt + (__bfloat162float(__float2bfloat16_rn(pmax)) - pmax);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars[L::kBarPFull + i]);

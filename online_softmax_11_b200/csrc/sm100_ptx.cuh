@@ -44,14 +44,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// One potentially blocking test of a phase.  The suspend-time hint lets the hardware park
+// the waiting warp until the phase completes (or about 0.5 ms pass) instead of having it
+// re-issue the test, so waiting warps leave the issue slots to the working ones.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "n"(500000)
       : "memory");
   return done != 0;
 }
@@ -66,21 +69,22 @@ struct WaitCtl {
 // Wait for the phase with parity `parity` of `bar` to complete.  Returns false (after
 // recording FA_ERR_TIMEOUT in g_status and raising the CTA's abort flag) when the wait
 // takes longer than ctl.limit_ns, or when another thread of the CTA has aborted.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl ctl) {
-  const uint32_t a = smem_addr(bar);
-  if (mbar_try_wait(a, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, const WaitCtl ctl) {
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(a, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (*ctl.abort) return false;
-      if (global_timer_ns() - t0 > ctl.limit_ns) {
-        *ctl.abort = 1;
-        atomicExch(&g_status, -7 /* FA_ERR_TIMEOUT */);
-        return false;
-      }
+    if (*ctl.abort) return false;
+    if (global_timer_ns() - t0 > ctl.limit_ns) {
+      *ctl.abort = 1;
+      atomicExch(&g_status, -7 /* FA_ERR_TIMEOUT */);
+      return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl ctl) {
+  const uint32_t a = smem_addr(bar);
+  if (mbar_try_wait(a, parity)) return true;  // common case: no call, no timer read
+  return mbar_wait_slow(a, parity, ctl);
 }
 
 // ---------------------------------------------------------------------------------
