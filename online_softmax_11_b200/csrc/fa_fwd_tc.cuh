@@ -183,7 +183,7 @@ __device__ __forceinline__ float2 tanh_small_pair(float2 x) {
 
 // How P is produced from the scores of one tile (chosen per tile, warp-uniformly).
 enum class PMode {
-  kPlainMixed,   // no soft-cap, no masked key: 7 of 8 pairs on ex2, 1 of 8 on the FMA pipe
+  kPlainMixed,   // no soft-cap, no masked key: 3 of 4 pairs on ex2, 1 of 4 on the FMA pipe
   kPlainMufu,    // no soft-cap, masked keys present (-inf -> exactly 0): all pairs on ex2
   kCapShort,     // soft-cap, every |s * scale / cap| < 0.12
   kCapLong,      // soft-cap, every |s * scale / cap| < 0.3
@@ -208,7 +208,7 @@ __device__ __forceinline__ float make_p(const float (&s)[kHalf], uint32_t taddr_
       float2 e;
       if constexpr (kMode == PMode::kPlainMixed || kMode == PMode::kPlainMufu) {
         const float2 u = __ffma2_rn(sv, make_float2(scale_log2, scale_log2), negm);
-        if (kMode == PMode::kPlainMixed && (x & 7) == 7)
+        if (kMode == PMode::kPlainMixed && (x & 3) == 3)  // one pair in four on the FMA pipe
           e = exp2_fma_pair(u);
         else
           e = ex2_pair(u);
@@ -513,13 +513,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c_lo = p.window > 0 ? max(0, row - p.window + 1 - k0) : 0;
 
         // Pass 1: row maximum (and minimum, for the soft-cap range check) over the two
-        // 64-score halves (four chains of three-input max), and the maximum of the
-        // columns whose exp2 runs on the FMA pipe in unmasked plain tiles (pairs 7 and 15
-        // of each 32-column chunk), to recompute the tile maximum's P with the very
-        // arithmetic that produced it.
-        float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F, mx2 = -CUDART_INF_F, mx3 = -CUDART_INF_F;
+        // 64-score halves with three-input max: three chains over the columns whose exp2
+        // runs on the MUFU in unmasked plain tiles, one over those on the FMA pipe (pair 3
+        // of every 4, i.e. columns 8k+6, 8k+7), so the tile maximum's P can be recomputed
+        // with the very arithmetic that produced it.
+        float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F, mx2 = -CUDART_INF_F, mx_emu = -CUDART_INF_F;
         float mn0 = CUDART_INF_F, mn1 = CUDART_INF_F;
-        float mx_emu = -CUDART_INF_F;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float s[kHalf];
@@ -529,10 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mx0 = fmax3(mx0, s[c], s[c + 1]);
             mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
             mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
-            mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+            mx_emu = fmax3(mx_emu, s[c + 6], s[c + 7]);
           }
-          mx_emu = fmax3(mx_emu, fmax3(s[14], s[15], s[30]), fmax3(s[31], s[46], s[47]));
-          mx_emu = fmax3(mx_emu, s[62], s[63]);
           if (p.use_softcap) {
 #pragma unroll
             for (int c = 0; c < kHalf; c += 4) {
@@ -541,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        const float mx = fmax3(fmaxf(mx0, mx1), mx2, mx3);
+        const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx_emu));
         const float mn = fminf(mn0, mn1);
         float m_tile;
         if (p.use_softcap)
