@@ -46,6 +46,8 @@
 #ifndef FA_SM100_H_
 #define FA_SM100_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -59,6 +61,9 @@ extern "C" {
 #define FA_ERR_BAD_ARG (-5)     /* scale not finite or <= 0, softcap not finite          */
 #define FA_ERR_CUDA (-6)        /* a CUDA runtime/driver call failed: fa_last_cuda_error */
 #define FA_ERR_TIMEOUT (-7)     /* a device-side wait exceeded its limit (see below)     */
+#define FA_ERR_WORKSPACE (-8)   /* split-KV workspace NULL, not 16-byte aligned or too small */
+
+#define FA_MAX_SPLITS 64        /* largest num_splits accepted by fa_fwd_splitkv          */
 
 /*
  * fa_fwd -- bf16 attention forward on the tensor cores (tcgen05 + TMA + TMEM).
@@ -78,6 +83,31 @@ extern "C" {
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
            int N, int d, float scale, int causal, int window, float softcap, void* stream);
+
+/*
+ * fa_fwd_splitkv -- the same operation as fa_fwd with the keys of every query row cut
+ * into num_splits contiguous chunks processed as separate work items (more parallelism
+ * for short sequences and few heads), then merged.  Chunk s yields a partial output O_s
+ * (normalised within the chunk) and LSE_s; the merge applies the two-block merge
+ * identities of "Module 16: Efficient and Long Attention", section 16.2, repeated over
+ * the chunks: with m = max_s LSE_s, weights w_s = exp(LSE_s - m), O = sum w_s O_s / sum w_s,
+ * LSE = m + ln sum w_s.  Same result as fa_fwd up to rounding.
+ *   num_splits : 1 .. FA_MAX_SPLITS.
+ *   workspace  : caller-owned DEVICE buffer of at least
+ *                fa_fwd_splitkv_workspace(B, Hq, N, d, num_splits) bytes, 16-byte aligned:
+ *                fp32 partial outputs [num_splits][B*Hq][N][d] followed by fp32 partial
+ *                LSE [num_splits][B*Hq][N].  Overwritten; no state kept between calls.
+ *                Calls that share one workspace must not overlap on the GPU.
+ *   Other arguments as fa_fwd.  FA_ERR_WORKSPACE if the workspace is missing, misaligned
+ *   or too small; FA_ERR_BAD_ARG for num_splits outside 1 .. FA_MAX_SPLITS.
+ */
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                   int N, int d, float scale, int causal, int window, float softcap, int num_splits,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* fa_fwd_splitkv_workspace -- bytes of workspace fa_fwd_splitkv needs (0 for an empty or
+ * invalid problem): num_splits * B * Hq * N * (d + 1) * 4. */
+size_t fa_fwd_splitkv_workspace(int B, int Hq, int N, int d, int num_splits);
 
 /*
  * fa_fwd_f32 -- the same operation in fp32 on the CUDA cores (FFMA, no TF32), for

@@ -30,10 +30,12 @@ ERRORS = {
     -5: "FA_ERR_BAD_ARG",
     -6: "FA_ERR_CUDA",
     -7: "FA_ERR_TIMEOUT",
+    -8: "FA_ERR_WORKSPACE",
 }
+MAX_SPLITS = 64
 # every symbol include/fa.h declares
-EXPORTS = ["fa_fwd", "fa_fwd_f32", "fa_check_status", "fa_selftest_wait_timeout", "fa_strerror",
-           "fa_last_cuda_error", "fa_version"]
+EXPORTS = ["fa_fwd", "fa_fwd_f32", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace", "fa_check_status",
+           "fa_selftest_wait_timeout", "fa_strerror", "fa_last_cuda_error", "fa_version"]
 
 _lock = threading.Lock()
 _lib = None
@@ -68,6 +70,10 @@ def load():
             fn = getattr(lib, name)
             fn.restype = i
             fn.argtypes = sig
+        lib.fa_fwd_splitkv.restype = i
+        lib.fa_fwd_splitkv.argtypes = sig[:-1] + [i, vp, ctypes.c_size_t, vp]
+        lib.fa_fwd_splitkv_workspace.restype = ctypes.c_size_t
+        lib.fa_fwd_splitkv_workspace.argtypes = [i, i, i, i, i]
         lib.fa_check_status.restype = i
         lib.fa_check_status.argtypes = [vp]
         lib.fa_selftest_wait_timeout.restype = i
@@ -135,6 +141,44 @@ def forward(q, k, v, *, scale: float | None = None, causal: bool = False, window
     return (out, lse) if return_lse else out
 
 
+def splitkv_workspace_bytes(B: int, Hq: int, N: int, d: int, num_splits: int) -> int:
+    """Workspace bytes ``fa_fwd_splitkv`` needs."""
+    return int(load().fa_fwd_splitkv_workspace(B, Hq, N, d, num_splits))
+
+
+def forward_splitkv(q, k, v, *, num_splits: int, scale: float | None = None, causal: bool = False,
+                    window: int = 0, softcap: float = 0.0, out=None, lse=None, workspace=None, stream=None):
+    """Split-KV attention forward (bf16) through ``fa_fwd_splitkv``; the workspace is a
+    caller tensor (allocated here with torch when not given)."""
+    import torch
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("fa_fwd_splitkv takes bfloat16 q, k, v")
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, N, d] with q's B, N and d")
+    for t in (q, k, v):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    if scale is None:
+        scale = float(torch.tensor(1.0, dtype=torch.float32) / torch.sqrt(torch.tensor(float(d), dtype=torch.float32)))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    need = splitkv_workspace_bytes(B, Hq, N, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        rc = load().fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq,
+                                   Hkv, N, d, float(scale), int(bool(causal)), int(window), float(softcap),
+                                   int(num_splits), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                   _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, load(), "fa_fwd_splitkv")
+    return out, lse
+
+
 def check_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return load().fa_check_status(_stream_handle(stream))
@@ -156,5 +200,5 @@ def attention_flops(B: int, Hq: int, N: int, d: int, causal: bool = False, windo
     return 4.0 * d * B * Hq * pairs
 
 
-__all__ = ["forward", "fwd_raw", "load", "check_status", "selftest_wait_timeout", "attention_flops", "FAError",
-           "EXPORTS", "LIB_PATH"]
+__all__ = ["forward", "forward_splitkv", "splitkv_workspace_bytes", "fwd_raw", "load", "check_status",
+           "selftest_wait_timeout", "attention_flops", "FAError", "EXPORTS", "LIB_PATH", "MAX_SPLITS"]

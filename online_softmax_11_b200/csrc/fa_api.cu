@@ -11,6 +11,7 @@
 #include "fa.h"
 #include "fa_fwd_f32.cuh"
 #include "fa_fwd_tc.cuh"
+#include "fa_merge.cuh"
 
 namespace {
 
@@ -57,10 +58,16 @@ int prepare_device(int dev, int* num_sms = nullptr) {
     }
     st.num_sms = prop.multiProcessorCount;
 
-    e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fa::tc::Layout<128>::kSmemLaunch);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::tc::Layout<64>::kSmemLaunch);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::tc::Layout<128>::kSmemLaunch);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                fa::tc::Layout<64>::kSmemLaunch);
     // the fp32 path needs up to 4 * (32 d + 32 (d + 1) + 32 d) bytes = 49280 at d = 128
     const int f32_smem = 64 * 1024;
@@ -148,18 +155,21 @@ const char* fa_strerror(int code) {
     case FA_ERR_BAD_ARG: return "scale must be finite and > 0, softcap finite";
     case FA_ERR_CUDA: return "CUDA call failed (see fa_last_cuda_error)";
     case FA_ERR_TIMEOUT: return "a device-side wait exceeded its limit";
+    case FA_ERR_WORKSPACE: return "workspace missing, misaligned or smaller than fa_fwd_splitkv_workspace()";
     default: return "unknown error code";
   }
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d,
-           float scale, int causal, int window, float softcap, void* stream) {
-  int rc = check_common(q, k, v, o, B, Hq, Hkv, N, d, scale, causal, window, softcap);
-  if (rc == 1) return FA_OK;
-  if (rc != FA_OK) return rc;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4)))
-    return FA_ERR_ALIGN;
+}  // extern "C"
+
+namespace {
+
+// Launch the tensor-core kernel: plain (num_splits == 0: bf16 O and fp32 LSE) or split-KV
+// (num_splits >= 1: fp32 partials into o_part / lse_part, then the merge kernel).
+int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+              int d, float scale, int causal, int window, float softcap, int num_splits, float* o_part,
+              float* lse_part, cudaStream_t s) {
+  int rc;
   int dev, num_sms = 0;
   if ((rc = current_device(&dev)) != FA_OK) return rc;
   if ((rc = prepare_device(dev, &num_sms)) != FA_OK) return rc;
@@ -170,6 +180,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   if ((rc = make_map(&mv, v, B * Hkv, N, d)) != FA_OK) return rc;
 
   namespace tc = fa::tc;
+  const bool split = num_splits >= 1;
   tc::Params p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -186,23 +197,87 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.cap_inner = softcap > 0.f ? scale / softcap : 0.f;
   p.cap_outer = softcap > 0.f ? softcap * tc::kLog2e : 0.f;
   p.timeout_ns = kWaitLimitNs;
+  p.num_splits = split ? num_splits : 1;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
 
-  const long long units = static_cast<long long>(B) * Hq * p.units_per_head;
+  const long long units = split ? static_cast<long long>(B) * Hq * p.n_qp * num_splits
+                                : static_cast<long long>(B) * Hq * p.units_per_head;
   if (units > 0x7fffffffll) return FA_ERR_BAD_SHAPE;
   p.n_units = static_cast<int>(units);
   // persistent: one CTA per SM (never more CTAs than units)
-  const long long grid = units < num_sms ? units : num_sms;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
   if (d == 128) {
-    tc::fa_fwd_tc_kernel<128><<<static_cast<unsigned>(grid), tc::kThreads, tc::Layout<128>::kSmemLaunch, s>>>(
-        mq, mk, mv, p);
+    if (split)
+      tc::fa_fwd_tc_kernel<128, true><<<grid, tc::kThreads, tc::Layout<128>::kSmemLaunch, s>>>(mq, mk, mv, p);
+    else
+      tc::fa_fwd_tc_kernel<128, false><<<grid, tc::kThreads, tc::Layout<128>::kSmemLaunch, s>>>(mq, mk, mv, p);
   } else {
-    tc::fa_fwd_tc_kernel<64><<<static_cast<unsigned>(grid), tc::kThreads, tc::Layout<64>::kSmemLaunch, s>>>(
-        mq, mk, mv, p);
+    if (split)
+      tc::fa_fwd_tc_kernel<64, true><<<grid, tc::kThreads, tc::Layout<64>::kSmemLaunch, s>>>(mq, mk, mv, p);
+    else
+      tc::fa_fwd_tc_kernel<64, false><<<grid, tc::kThreads, tc::Layout<64>::kSmemLaunch, s>>>(mq, mk, mv, p);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
+  if (split) {
+    const long long rows = static_cast<long long>(B) * Hq * N;
+    const unsigned mgrid = static_cast<unsigned>((rows + fa::kMergeRowsPerBlock - 1) / fa::kMergeRowsPerBlock);
+    if (d == 128)
+      fa::fa_merge_splits_kernel<128><<<mgrid, 32 * fa::kMergeRowsPerBlock, 0, s>>>(
+          o_part, lse_part, static_cast<__nv_bfloat16*>(o), lse, rows, num_splits);
+    else
+      fa::fa_merge_splits_kernel<64><<<mgrid, 32 * fa::kMergeRowsPerBlock, 0, s>>>(
+          o_part, lse_part, static_cast<__nv_bfloat16*>(o), lse, rows, num_splits);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   return FA_OK;
+}
+
+int check_bf16(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int Hq, int Hkv,
+               int N, int d, float scale, int causal, int window, float softcap) {
+  int rc = check_common(q, k, v, o, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+  if (rc != FA_OK) return rc;  // 1 = empty problem
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4)))
+    return FA_ERR_ALIGN;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d,
+           float scale, int causal, int window, float softcap, void* stream) {
+  int rc = check_bf16(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  return launch_tc(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap, 0, nullptr, nullptr,
+                   static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_fwd_splitkv_workspace(int B, int Hq, int N, int d, int num_splits) {
+  if (B <= 0 || Hq <= 0 || N <= 0 || d <= 0 || num_splits < 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * Hq * N;
+  return static_cast<size_t>(num_splits) * rows * (static_cast<size_t>(d) + 1) * sizeof(float);
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                   int d, float scale, int causal, int window, float softcap, int num_splits, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  int rc = check_bf16(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (num_splits < 1 || num_splits > FA_MAX_SPLITS) return FA_ERR_BAD_ARG;
+  const size_t need = fa_fwd_splitkv_workspace(B, Hq, N, d, num_splits);
+  if (workspace == nullptr || !aligned(workspace, 16) || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  const size_t rows = static_cast<size_t>(B) * Hq * N;
+  float* o_part = static_cast<float*>(workspace);
+  float* lse_part = o_part + static_cast<size_t>(num_splits) * rows * d;
+  return launch_tc(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap, num_splits, o_part, lse_part,
+                   static_cast<cudaStream_t>(stream));
 }
 
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Hq, int Hkv, int N,

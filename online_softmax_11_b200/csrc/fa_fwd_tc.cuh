@@ -117,6 +117,12 @@ struct Params {
   float cap_inner;     // scale / softcap
   float cap_outer;     // softcap * log2(e)
   unsigned long long timeout_ns;
+  // split-KV: the key tiles of every query-tile pair are cut into num_splits contiguous
+  // chunks, each chunk a work tile of its own, writing a partial O (fp32, normalised
+  // within the chunk) and a partial LSE for a merge pass (fa_merge.cuh)
+  int num_splits;      // 1: plain forward, outputs o / lse
+  float* o_part;       // [num_splits][B*Hq][N][d]
+  float* lse_part;     // [num_splits][B*Hq][N]
 };
 
 // Accurate tanh for the soft-cap: Taylor series about 0 through x^11 for |x| < 0.3
@@ -251,7 +257,8 @@ __device__ __forceinline__ void load_half(uint32_t taddr, int c0, bool need_mask
 struct TileRange {
   int r0, r1;  // first / last query row (r1 < N)
   int lo, hi;
-  bool active;
+  bool active;  // the tile has rows below N
+  bool part;    // ... and key tiles to process in this work tile (lo < hi)
 };
 
 __device__ __forceinline__ TileRange tile_range(int r0, int N, int nkv, int causal, int window) {
@@ -264,53 +271,87 @@ __device__ __forceinline__ TileRange tile_range(int r0, int N, int nkv, int caus
   if (causal) t.hi = min(nkv, t.r1 / BN + 1);
   if (window > 0) t.lo = max(0, t.r0 - window + 1) / BN;
   if (!t.active) t.lo = t.hi = 0;
+  t.part = t.active && t.lo < t.hi;
   return t;
 }
 
 __device__ __forceinline__ bool participates(const TileRange& t, int j) { return t.active && j >= t.lo && j < t.hi; }
 
-// One work tile: (batch*head, query-tile pair) and the key tiles it streams.
+// One work tile: (batch*head, query-tile pair, key chunk) and the key tiles it streams.
 struct WorkTile {
   int bh, kvh;
+  int split;   // key chunk (0 without split-KV)
   TileRange tr0, tr1;
-  int lo, hi;  // union key-tile range
+  int lo, hi;  // union key-tile range of the participating query tiles
   __device__ const TileRange& tr(int i) const { return i == 0 ? tr0 : tr1; }
 };
 
-__device__ __forceinline__ WorkTile make_work_tile(const Params& p, int bh, int qp) {
+__device__ __forceinline__ void clip(TileRange& t, int jlo, int jhi) {
+  t.lo = max(t.lo, jlo);
+  t.hi = min(t.hi, jhi);
+  t.part = t.active && t.lo < t.hi;
+  if (!t.part) t.lo = t.hi = 0;
+}
+
+__device__ __forceinline__ WorkTile make_work_tile(const Params& p, int bh, int qp, int split) {
   WorkTile w;
   w.bh = bh;
+  w.split = split;
   const int b = bh / p.Hq;
   const int hq = bh - b * p.Hq;
   w.kvh = b * p.Hkv + hq / (p.Hq / p.Hkv);
   const int nkv = (p.N + BN - 1) / BN;
   w.tr0 = tile_range(qp * NQ * BM, p.N, nkv, p.causal, p.window);
   w.tr1 = tile_range(qp * NQ * BM + BM, p.N, nkv, p.causal, p.window);
-  w.lo = w.tr0.lo;
-  w.hi = w.tr0.hi;
+  int ulo = w.tr0.lo, uhi = w.tr0.hi;
   if (w.tr1.active) {
-    w.lo = min(w.lo, w.tr1.lo);
+    ulo = min(ulo, w.tr1.lo);
+    uhi = max(uhi, w.tr1.hi);
+  }
+  if (p.num_splits > 1) {  // this work tile keeps chunk `split` of the pair's key tiles
+    const int T = uhi - ulo;
+    const int jlo = ulo + (split * T) / p.num_splits;
+    const int jhi = ulo + ((split + 1) * T) / p.num_splits;
+    clip(w.tr0, jlo, jhi);
+    clip(w.tr1, jlo, jhi);
+  }
+  w.lo = w.hi = 0;
+  if (w.tr0.part) {
+    w.lo = w.tr0.lo;
+    w.hi = w.tr0.hi;
+  }
+  if (w.tr1.part) {
+    w.lo = w.tr0.part ? min(w.lo, w.tr1.lo) : w.tr1.lo;
     w.hi = max(w.hi, w.tr1.hi);
   }
   return w;
 }
 
-// The static schedule: CTA c takes units c, c + G, ...; unit u is head u / U, pair index
-// p = u % U, and covers q-pairs n_qp-1-p (longer under causal) and p (when distinct).
+// The static schedule: CTA c takes units c, c + G, ....  Without split-KV, unit u is head
+// u / U, pair index p = u % U, and covers q-pairs n_qp-1-p (longer under causal) and p
+// (when distinct).  With split-KV, unit u is (head, q-pair from the longest, key chunk).
 // Every role walks the same sequence; the callback returns false to stop (abort).
 template <typename F>
 __device__ __forceinline__ void for_each_tile(const Params& p, F&& f) {
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    if (p.num_splits > 1) {
+      const int per_head = p.n_qp * p.num_splits;
+      const int bh = u / per_head;
+      const int rem = u - bh * per_head;
+      const int qp = p.n_qp - 1 - rem / p.num_splits;
+      if (!f(make_work_tile(p, bh, qp, rem % p.num_splits))) return;
+      continue;
+    }
     const int bh = u / p.units_per_head;
     const int pi = u - bh * p.units_per_head;
     const int qa = p.n_qp - 1 - pi;
     for (int half = 0; half < (pi != qa ? 2 : 1); ++half) {  // one call site: f inlines once
-      if (!f(make_work_tile(p, bh, half == 0 ? qa : pi))) return;
+      if (!f(make_work_tile(p, bh, half == 0 ? qa : pi, 0))) return;
     }
   }
 }
 
-template <int D>
+template <int D, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -366,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < NQ; ++i) {
           const TileRange& t = w.tr(i);
-          if (!t.active) continue;
+          if (!t.part) continue;
           if (!mbar_wait(&bars[L::kBarQEmpty + i], (q_cnt[i] & 1u) ^ 1u, ctl)) return false;
           mbar_arrive_expect_tx(&bars[L::kBarQFull + i], L::kTileBytes);
           for (int h = 0; h < L::kHalves; ++h)
@@ -490,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for_each_tile(p, [&](const WorkTile& w) {
       const TileRange& t = w.tr(i);
-      if (!t.active) return true;
+      if (!t.active) return true;  // rows past N: nothing to write
       const int row = t.r0 + trow;
       float m = -CUDART_INF_F;  // running reference maximum (log2 units)
       float l = 0.f;            // running sum of P (fp32) relative to m
@@ -624,11 +665,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         o_valid = true;
       }
 
-      // ---- epilogue: O / lr -> bf16, LSE = (m + log2 l) ln 2
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarOFull + i], o_phase, ctl))) return false;
-      o_phase ^= 1u;
-      tc_fence_after();
+      // ---- epilogue: O / lr -> bf16, LSE = (m + log2 l) ln 2 (split-KV: fp32 partials;
+      // a query tile with no key tile in this chunk writes O = 0 and LSE = -inf)
+      if (t.part) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarOFull + i], o_phase, ctl))) return false;
+        o_phase ^= 1u;
+        tc_fence_after();
+      }
       const float inv = lr > 0.f ? 1.0f / lr : 0.f;
+      if constexpr (kSplit) {
+        const int64_t prow = (static_cast<int64_t>(w.split) * p.n_bh + w.bh) * p.N + row;
+        float* orow = p.o_part + prow * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          if (t.part) {
+            tmem_ld32_wait(lane_base + colO + c * 32, r);
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) r[x] = 0u;
+          }
+          if (row < p.N) {
+            float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              dst[x] = make_float4(__uint_as_float(r[4 * x]) * inv, __uint_as_float(r[4 * x + 1]) * inv,
+                                   __uint_as_float(r[4 * x + 2]) * inv, __uint_as_float(r[4 * x + 3]) * inv);
+          }
+        }
+        if (row < p.N) p.lse_part[prow] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+        return true;
+      }
       __nv_bfloat16* orow = p.o + (static_cast<int64_t>(w.bh) * p.N + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {

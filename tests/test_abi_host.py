@@ -107,3 +107,29 @@ def test_build_command_targets_sm100a_only():
     cmd = fabuild.command()
     assert "arch=compute_100a,code=sm_100a" in cmd
     assert not any("sm_90" in c or "sm_80" in c for c in cmd)
+
+
+def call_split(lib, num_splits=2, ws=FAKE, ws_bytes=1 << 30, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, N=8, d=64, scale=0.125, causal=0,
+             window=0, softcap=0.0)
+    a.update(kw)
+    return lib.fa_fwd_splitkv(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"],
+                              a["scale"], a["causal"], a["window"], a["softcap"], num_splits, ws, ws_bytes, None)
+
+
+def test_splitkv_workspace_size(lib):
+    # num_splits x rows x (d + 1) floats
+    assert lib.fa_fwd_splitkv_workspace(2, 3, 5, 64, 4) == 4 * 2 * 3 * 5 * 65 * 4
+    assert lib.fa_fwd_splitkv_workspace(0, 3, 5, 64, 4) == 0
+    assert lib.fa_fwd_splitkv_workspace(1, 1, 1, 128, 0) == 0
+
+
+def test_splitkv_argument_errors(lib):
+    assert call_split(lib, num_splits=0) == -5
+    assert call_split(lib, num_splits=fa.MAX_SPLITS + 1) == -5
+    assert call_split(lib, ws=None) == -8
+    assert call_split(lib, ws=FAKE + 4) == -8
+    assert call_split(lib, ws_bytes=16) == -8
+    assert call_split(lib, d=32) == -3
+    assert call_split(lib, Hq=3) == -2
+    assert call_split(lib, q=None, k=None, v=None, o=None, lse=None, ws=None, N=0) == 0  # empty problem
