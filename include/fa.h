@@ -63,7 +63,11 @@ extern "C" {
 #define FA_ERR_TIMEOUT (-7)     /* a device-side wait exceeded its limit (see below)     */
 #define FA_ERR_WORKSPACE (-8)   /* split-KV workspace NULL, not 16-byte aligned or too small */
 
+#define FA_ERR_SCRATCH_LIMIT (-9) /* fa_fwd_splitkv_static: problem too large for the fixed
+                                     scratch array (see FA_STATIC_SCRATCH_BYTES)           */
+
 #define FA_MAX_SPLITS 64        /* largest num_splits accepted by fa_fwd_splitkv          */
+#define FA_STATIC_SCRATCH_BYTES (32u << 20) /* scratch array of fa_fwd_splitkv_static     */
 
 /*
  * fa_fwd -- bf16 attention forward on the tensor cores (tcgen05 + TMA + TMEM).
@@ -108,6 +112,35 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
 /* fa_fwd_splitkv_workspace -- bytes of workspace fa_fwd_splitkv needs (0 for an empty or
  * invalid problem): num_splits * B * Hq * N * (d + 1) * 4. */
 size_t fa_fwd_splitkv_workspace(int B, int Hq, int N, int d, int num_splits);
+
+/*
+ * fa_fwd_splitkv_static -- fa_fwd_splitkv for callers that cannot allocate device memory.
+ * The reference pages have no counterpart to this entry point; it is a deployment
+ * convenience of this library.
+ *
+ * Some callers have no way to obtain a workspace: a host program that runs under a fixed
+ * device-memory plan where nothing may call cudaMalloc after start-up (cudaMalloc and
+ * cudaFree can also synchronise the device, which latency-bound callers avoid), or a
+ * plug-in inside a framework that owns all device memory through its own allocator and
+ * offers no scratch to plug-ins.  This entry point takes no workspace and allocates
+ * nothing (no cudaMalloc, no cudaFree, no allocating library call): its scratch is a
+ * fixed array of FA_STATIC_SCRATCH_BYTES (32 MiB) compiled into the library, which every
+ * GPU the library is loaded on holds until the process exits.
+ *   Arguments: as fa_fwd_splitkv without workspace / workspace_bytes.  The caller still
+ *   owns q, k, v, o and lse.
+ *   Limit: problems whose fa_fwd_splitkv_workspace(B, Hq, N, d, num_splits) exceeds
+ *   FA_STATIC_SCRATCH_BYTES are rejected with FA_ERR_SCRATCH_LIMIT (nothing is written).
+ *   Set-up: the first call on a device, with that device current, looks up the array's
+ *   device address (cudaGetSymbolAddress) once; make that first call before any stream
+ *   capture is begun on the device.
+ *   Sharing: every call on a device uses the same array, and the array keeps the last
+ *   call's partial results.  Nothing in it has to start at zero (each call writes every
+ *   partial it reads), but calls that overlap on the GPU (on different streams, or from
+ *   different host threads) race on the array: serialise them.
+ */
+int fa_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                          int Hkv, int N, int d, float scale, int causal, int window, float softcap,
+                          int num_splits, void* stream);
 
 /*
  * fa_fwd_f32 -- the same operation in fp32 on the CUDA cores (FFMA, no TF32), for

@@ -31,11 +31,13 @@ ERRORS = {
     -6: "FA_ERR_CUDA",
     -7: "FA_ERR_TIMEOUT",
     -8: "FA_ERR_WORKSPACE",
+    -9: "FA_ERR_SCRATCH_LIMIT",
 }
+STATIC_SCRATCH_BYTES = 32 << 20
 MAX_SPLITS = 64
 # every symbol include/fa.h declares
-EXPORTS = ["fa_fwd", "fa_fwd_f32", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace", "fa_check_status",
-           "fa_selftest_wait_timeout", "fa_strerror", "fa_last_cuda_error", "fa_version"]
+EXPORTS = ["fa_fwd", "fa_fwd_f32", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace", "fa_fwd_splitkv_static",
+           "fa_check_status", "fa_selftest_wait_timeout", "fa_strerror", "fa_last_cuda_error", "fa_version"]
 
 _lock = threading.Lock()
 _lib = None
@@ -72,6 +74,8 @@ def load():
             fn.argtypes = sig
         lib.fa_fwd_splitkv.restype = i
         lib.fa_fwd_splitkv.argtypes = sig[:-1] + [i, vp, ctypes.c_size_t, vp]
+        lib.fa_fwd_splitkv_static.restype = i
+        lib.fa_fwd_splitkv_static.argtypes = sig[:-1] + [i, vp]
         lib.fa_fwd_splitkv_workspace.restype = ctypes.c_size_t
         lib.fa_fwd_splitkv_workspace.argtypes = [i, i, i, i, i]
         lib.fa_check_status.restype = i

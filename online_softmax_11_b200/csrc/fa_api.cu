@@ -156,6 +156,8 @@ const char* fa_strerror(int code) {
     case FA_ERR_CUDA: return "CUDA call failed (see fa_last_cuda_error)";
     case FA_ERR_TIMEOUT: return "a device-side wait exceeded its limit";
     case FA_ERR_WORKSPACE: return "workspace missing, misaligned or smaller than fa_fwd_splitkv_workspace()";
+    case FA_ERR_SCRATCH_LIMIT:
+      return "problem needs more split-KV scratch than fa_fwd_splitkv_static's fixed array (FA_STATIC_SCRATCH_BYTES)";
     default: return "unknown error code";
   }
 }
@@ -312,6 +314,68 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return FA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// split-KV without a caller workspace
+// ---------------------------------------------------------------------------------
+namespace {
+
+// Scratch of fa_fwd_splitkv_static: a fixed array in this library's device image.  Every
+// GPU the library is loaded on holds it until the process exits.  In host code its name
+// only stands in for the symbol; the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_splitkv_scratch[FA_STATIC_SCRATCH_BYTES];
+
+struct ScratchState {
+  std::once_flag once;
+  int status = FA_OK;
+  void* ptr = nullptr;
+};
+ScratchState g_scratch[kMaxDevices];
+
+// Device address of the scratch array on device `dev` (the current device): looked up
+// once per device, on the first call made with that device current.
+int scratch_address(int dev, void** out) {
+  ScratchState& st = g_scratch[dev];
+  std::call_once(st.once, [&] {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_splitkv_scratch);
+    if (e != cudaSuccess) {
+      st.status = cuda_fail(e);
+      return;
+    }
+    st.ptr = ptr;
+  });
+  *out = st.ptr;
+  return st.status;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                          int N, int d, float scale, int causal, int window, float softcap, int num_splits,
+                          void* stream) {
+  int rc = check_bf16(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (num_splits < 1 || num_splits > FA_MAX_SPLITS) return FA_ERR_BAD_ARG;
+  const size_t need = fa_fwd_splitkv_workspace(B, Hq, N, d, num_splits);
+  if (need > static_cast<size_t>(FA_STATIC_SCRATCH_BYTES)) return FA_ERR_SCRATCH_LIMIT;
+  int dev;
+  if ((rc = current_device(&dev)) != FA_OK) return rc;
+  void* scratch = nullptr;
+  if ((rc = scratch_address(dev, &scratch)) != FA_OK) return rc;
+  // Every partial the merge reads is written earlier in the same call (each chunk writes
+  // O and LSE for every row, -inf / 0 where it has no keys), so nothing has to be cleared.
+  const size_t rows = static_cast<size_t>(B) * Hq * N;
+  float* o_part = static_cast<float*>(scratch);
+  float* lse_part = o_part + static_cast<size_t>(num_splits) * rows * d;
+  return launch_tc(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap, num_splits, o_part, lse_part,
+                   static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
