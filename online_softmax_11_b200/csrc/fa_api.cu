@@ -203,8 +203,10 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.o_part = o_part;
   p.lse_part = lse_part;
 
-  const long long units = split ? static_cast<long long>(B) * Hq * p.n_qp * num_splits
-                                : static_cast<long long>(B) * Hq * p.units_per_head;
+  // the kernel walks split units (head, q-pair, chunk) only for more than one chunk; a
+  // single chunk keeps the paired schedule of the plain forward (for_each_tile)
+  const long long units = p.num_splits > 1 ? static_cast<long long>(B) * Hq * p.n_qp * p.num_splits
+                                           : static_cast<long long>(B) * Hq * p.units_per_head;
   if (units > 0x7fffffffll) return FA_ERR_BAD_SHAPE;
   p.n_units = static_cast<int>(units);
   // persistent: one CTA per SM (never more CTAs than units)

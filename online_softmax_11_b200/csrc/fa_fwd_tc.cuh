@@ -337,12 +337,14 @@ __device__ __forceinline__ void for_each_tile(const Params& p, F&& f) {
     if (p.num_splits > 1) {
       const int per_head = p.n_qp * p.num_splits;
       const int bh = u / per_head;
+      if (bh >= p.n_bh) return;  // never past the last head, whatever n_units says
       const int rem = u - bh * per_head;
       const int qp = p.n_qp - 1 - rem / p.num_splits;
       if (!f(make_work_tile(p, bh, qp, rem % p.num_splits))) return;
       continue;
     }
     const int bh = u / p.units_per_head;
+    if (bh >= p.n_bh) return;
     const int pi = u - bh * p.units_per_head;
     const int qa = p.n_qp - 1 - pi;
     for (int half = 0; half < (pi != qa ? 2 : 1); ++half) {  // one call site: f inlines once

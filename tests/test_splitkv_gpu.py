@@ -29,6 +29,8 @@ def fa():
 CASES = [
     # B, Hq, Hkv, N, d, causal, window, softcap, splits
     (1, 2, 2, 1, 128, False, 0, 0.0, 1),
+    (2, 4, 2, 1000, 64, True, 0, 0.0, 1),     # one chunk over several query-tile pairs
+    (1, 2, 2, 700, 128, False, 0, 0.0, 1),
     (1, 2, 2, 300, 128, False, 0, 0.0, 2),
     (2, 4, 2, 513, 64, False, 0, 0.0, 3),
     (1, 2, 2, 1000, 128, True, 0, 0.0, 4),
@@ -60,14 +62,14 @@ def test_splitkv_matches_oracle(fa, B, Hq, Hkv, N, d, causal, window, softcap, s
 
 
 def test_splitkv_full_size_d64_workload(fa):
-    """B=4 H=16 N=1024 d=64 with 2 and 4 chunks, compared on the standard row sample."""
+    """B=4 H=16 N=1024 d=64 with 1, 2 and 4 chunks, compared on the standard row sample."""
     w = workloads.WORKLOADS["mha_b4_h16_n1k_d64"]
     q, k, v = workloads.make_inputs(w)
     dev = torch.device("cuda:0")
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     rows = workloads.sample_rows(w, workloads.standard_row_sample(w.N), heads=[0, 17, 40, 63])
     ro, rlse = oracle.attention(q, k, v, scale=w.scale, rows=rows)
-    for splits in (2, 4):
+    for splits in (1, 2, 4):
         o, lse = fa.forward_splitkv(qd, kd, vd, num_splits=splits, scale=w.scale)
         torch.cuda.synchronize()
         assert fa.check_status() == 0
