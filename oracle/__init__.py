@@ -46,7 +46,7 @@ _lib = None
 DTYPE_CODES = {"float64": 0, "float32": 1, "bfloat16": 2}
 _ARGTYPES = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
              ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
-             ctypes.c_int64, ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_double,
+             ctypes.c_int64, ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
              ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
 
 
@@ -115,13 +115,15 @@ def _as_host_array(t):
     raise TypeError(f"oracle: unsupported dtype {a.dtype}")
 
 
-def attention(q, k, v, *, scale: float, causal: bool = False, window: int = 0,
+def attention(q, k, v, *, scale: float, causal: bool = False, window: int = 0, n_sink: int = 0,
               softcap: float = 0.0, rows=None, nthreads: int | None = None, _lib=None):
     """Dense fp64 attention.
 
     q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d] (torch or numpy; fp64, fp32 or bf16 — all
     three the same type).  Self-attention has Nq == Nk; with Nq < Nk the queries are the
     last Nq positions of the key sequence for the causal and window masks.
+    ``n_sink``: the first ``n_sink`` keys are attention sinks, exempt from the window
+    (Module 16, section 16.6); they stay under the causal mask.
     ``rows``: optional flat row indices ``(b*Hq + hq)*Nq + i``.
     Returns ``(O, LSE)`` as float64 numpy arrays: ``O[B,Hq,Nq,d]``, ``LSE[B,Hq,Nq]`` for
     all rows, or ``O[len(rows), d]``, ``LSE[len(rows)]`` for a row subset.
@@ -154,7 +156,7 @@ def attention(q, k, v, *, scale: float, causal: bool = False, window: int = 0,
     lib = _lib if _lib is not None else _load()
     rc = lib.oracle_attn_fp64(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, qt,
                                   B, Hq, Hkv, N, Nk, d, float(scale), int(bool(causal)), int(window),
-                                  float(softcap), rows_ptr, nrows, o.ctypes.data, lse.ctypes.data,
+                                  int(n_sink), float(softcap), rows_ptr, nrows, o.ctypes.data, lse.ctypes.data,
                                   int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_attn_fp64 failed with status {rc}")

@@ -23,9 +23,13 @@
  *   2. if softcap > 0:  s_j = softcap * tanh(s_j / softcap)
  *                                       (Module 16, section 16.5, logit soft-capping)
  *   3. with the query's position in the key sequence p = i + (Nk - Nq):
- *      s_j = -inf  if (causal and j > p) or (window > 0 and p - j >= window)
+ *      s_j = -inf  if (causal and j > p)
+ *                  or (window > 0 and p - j >= window and j >= n_sink)
  *                   (Module 16, 16.2 "Measured": the causal mask uses positions in the
- *                    full sequence; 16.3: a local layer sees the W most recent tokens).
+ *                    full sequence; 16.3: a local layer sees the W most recent tokens;
+ *                    16.6: the first tokens, the attention sinks, are kept alongside the
+ *                    sliding window -- they are exempt from the window, not from the
+ *                    causal mask, and n_sink = 0 is the plain window).
  *      With Nq == Nk (self-attention) p = i; with fewer queries than keys the queries
  *      are the last Nq positions of the key sequence (cross-attention / decode).
  *   4. m = max_j s_j,  p_j = exp(s_j - m),  l = sum_j p_j,
@@ -69,6 +73,7 @@ typedef struct {
   double scale;
   int causal;
   int64_t window;
+  int64_t n_sink;
   double softcap;
   const int64_t* rows; /* NULL: every row in order */
   int64_t nrows;
@@ -98,7 +103,7 @@ static void attend_row(const job_t* J, int64_t row, double* s, double* o_row, do
     double sj = J->scale * dot;
     if (J->softcap > 0.0) sj = J->softcap * tanh(sj / J->softcap);
     if (J->causal && j > pos) sj = -INFINITY;
-    if (J->window > 0 && pos - j >= J->window) sj = -INFINITY;
+    if (J->window > 0 && pos - j >= J->window && j >= J->n_sink) sj = -INFINITY;
     s[j] = sj;
   }
 
@@ -141,13 +146,14 @@ static void* worker(void* arg) {
  * oracle_attn_fp64 -- O and LSE for the listed query rows.
  *   rows[r] is a flat row index (b*Hq + hq)*Nq + i; rows == NULL means all B*Hq*Nq rows.
  *   o receives nrows*d doubles, lse nrows doubles, in the order of `rows`.
+ *   n_sink >= 0 keys at the start of the key sequence are exempt from the window.
  * Returns 0, or -1 for bad arguments, -2 when memory or threads could not be had.
  */
 int oracle_attn_fp64(const void* q, const void* k, const void* v, int dtype, int64_t B, int64_t Hq,
                      int64_t Hkv, int64_t Nq, int64_t Nk, int64_t d, double scale, int causal, int64_t window,
-                     double softcap, const int64_t* rows, int64_t nrows, double* o, double* lse,
+                     int64_t n_sink, double softcap, const int64_t* rows, int64_t nrows, double* o, double* lse,
                      int nthreads) {
-  if (B < 0 || Hq < 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0 || (Hq % Hkv) != 0) return -1;
+  if (B < 0 || Hq < 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0 || (Hq % Hkv) != 0 || n_sink < 0) return -1;
   if (dtype != ORACLE_F64 && dtype != ORACLE_F32 && dtype != ORACLE_BF16) return -1;
   int64_t total = B * Hq * Nq;
   if (!rows) nrows = total;
@@ -170,7 +176,7 @@ int oracle_attn_fp64(const void* q, const void* k, const void* v, int dtype, int
   int rc = 0;
   int started = 0;
   for (int t = 0; t < nthreads; ++t) {
-    job_t J = {q, k, v, dtype, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, softcap,
+    job_t J = {q, k, v, dtype, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, n_sink, softcap,
                rows, nrows, o, lse, nthreads, t, 0};
     jobs[t] = J;
   }

@@ -319,6 +319,98 @@ def pin_nx_modular(attn):
     assert np.max(np.abs(o - ro)) < 1e-12 and np.max(np.abs(lse - rlse)) < 1e-12
 
 
+def _kept_keys(pos, nk, causal, window, n_sink):
+    """The keys a query at position ``pos`` sees, built as sets from the section's words:
+    with a window, the ``window`` most recent tokens up to the query itself, together with
+    the first ``n_sink`` tokens (Module 16, 16.6), never a token after the query when
+    causal (16.2)."""
+    visible = set(range(nk)) if not causal else set(range(max(0, min(pos + 1, nk))))
+    if window <= 0:
+        return sorted(visible)
+    recent = set(range(max(0, pos - window + 1), pos + 1))
+    sinks = set(range(n_sink))
+    return sorted(visible & (recent | sinks))
+
+
+def pin_attention_sinks(attn):
+    """Attention sinks (Module 16, 16.6: the first tokens kept alongside the sliding
+    window).  (a) Against a library softmax over the key set built explicitly per row,
+    self- and cross-attention shapes, sinks fewer and more than the window, rows before
+    the sinks end; (b) no sinks is the plain window and sinks covering every key are
+    plain causal attention, bit for bit; (c) zero queries give LSE = ln(#kept keys) in
+    closed form; (d) a row whose sinks and window are disjoint is the block merge
+    (16.2) of attention over the sinks alone and over the window alone."""
+    cases = [  # Nq, Nk, d, window, n_sink, cap
+        (21, 21, 5, 4, 3, 0.0),
+        (21, 21, 4, 1, 4, 0.0),
+        (16, 16, 3, 6, 9, 2.0),
+        (7, 19, 6, 5, 2, 0.0),
+        (19, 19, 4, 3, 1, 0.0),
+    ]
+    for n, (nq, nk, d, window, n_sink, cap) in enumerate(cases):
+        q, k, v = _rand((1, 2, nq, d), 401 + n), _rand((1, 1, nk, d), 411 + n), _rand((1, 1, nk, d), 421 + n)
+        scale = 0.7
+        o, lse = attn(q, k, v, scale=scale, causal=True, window=window, n_sink=n_sink, softcap=cap)
+        for h in range(2):
+            for i in range(nq):
+                keep = _kept_keys(i + nk - nq, nk, True, window, n_sink)
+                s = torch.as_tensor(scale * (q[0, h, i] @ k[0, 0, keep].T))
+                if cap > 0:
+                    s = cap * torch.tanh(s / cap)
+                w = torch.softmax(s, dim=-1).numpy()
+                assert np.max(np.abs(o[0, h, i] - w @ v[0, 0, keep])) < 1e-12, (n, h, i)
+                assert abs(lse[0, h, i] - float(torch.logsumexp(s, dim=-1))) < 1e-12, (n, h, i)
+    # (b) limits
+    N, d = 18, 4
+    q, k, v = _rand((1, 2, N, d), 431), _rand((1, 2, N, d), 432), _rand((1, 2, N, d), 433)
+    oa, la = attn(q, k, v, scale=0.6, causal=True, window=5, n_sink=0)
+    ob, lb = attn(q, k, v, scale=0.6, causal=True, window=5)
+    assert np.array_equal(oa, ob) and np.array_equal(la, lb)
+    oa, la = attn(q, k, v, scale=0.6, causal=True, window=5, n_sink=N)
+    ob, lb = attn(q, k, v, scale=0.6, causal=True)
+    assert np.array_equal(oa, ob) and np.array_equal(la, lb)
+    # (c) uniform weights
+    for window, n_sink in [(4, 4), (1, 2), (6, 1)]:
+        o, lse = attn(np.zeros_like(q), k, v, scale=0.6, causal=True, window=window, n_sink=n_sink)
+        for i in range(N):
+            cnt = min(i + 1, window) + min(n_sink, max(0, i - window + 1))
+            assert abs(lse[0, 0, i] - math.log(cnt)) < 1e-12, (window, n_sink, i)
+    # (d) block merge of the sinks and the window
+    W, S = 4, 3
+    o, lse = attn(q, k, v, scale=0.6, causal=True, window=W, n_sink=S)
+    for i in range(S + W, N):
+        o1, l1 = attn(q[:, :, i:i + 1], k[:, :, :S], v[:, :, :S], scale=0.6)
+        o2, l2 = attn(q[:, :, i:i + 1], k[:, :, i - W + 1:i + 1], v[:, :, i - W + 1:i + 1], scale=0.6)
+        s = 0.6 * np.einsum("hd,hjd->hj", q[0, :, i], k[0])
+        m1, m2 = s[:, :S].max(-1), s[:, i - W + 1:i + 1].max(-1)
+        m, l, om = oracle.merge(m1, np.exp(l1[0, :, 0] - m1), o1[0, :, 0], m2, np.exp(l2[0, :, 0] - m2), o2[0, :, 0])
+        assert np.max(np.abs(om - o[0, :, i])) < 1e-12
+        assert np.max(np.abs(m + np.log(l) - lse[0, :, i])) < 1e-12
+
+
+def pin_cross_attention(attn):
+    """Fewer (or more) queries than keys: the queries are the last Nq positions of the
+    key sequence.  Non-causal cross-attention of one query row equals self-attention's
+    row over the same keys; causal rows equal the prefix attention at their global
+    position; with more queries than keys the rows before the first key see nothing
+    (O = 0, LSE = -inf, as the oxios routine leaves a row whose sum stays zero)."""
+    nk, d = 13, 4
+    k, v = _rand((1, 1, nk, d), 441), _rand((1, 1, nk, d), 442)
+    qs = _rand((1, 1, nk, d), 443)
+    o_self, l_self = attn(qs, k, v, scale=0.5, causal=True)
+    for nq in (1, 4, nk):
+        o, lse = attn(qs[:, :, nk - nq:], k, v, scale=0.5, causal=True)
+        assert np.array_equal(o[0, 0], o_self[0, 0, nk - nq:]) and np.array_equal(lse[0, 0], l_self[0, 0, nk - nq:])
+    o_full, l_full = attn(qs, k, v, scale=0.5)
+    o, lse = attn(qs[:, :, 5:6], k, v, scale=0.5)
+    assert np.array_equal(o[0, 0, 0], o_full[0, 0, 5]) and lse[0, 0, 0] == l_full[0, 0, 5]
+    qm = _rand((1, 1, nk + 3, d), 444)
+    o, lse = attn(qm, k, v, scale=0.5, causal=True)
+    assert np.all(o[0, 0, :3] == 0.0) and np.all(lse[0, 0, :3] == -np.inf)
+    ref, rl = attn(qm[:, :, 3:], k, v, scale=0.5, causal=True)
+    assert np.array_equal(o[0, 0, 3:], ref[0, 0]) and np.array_equal(lse[0, 0, 3:], rl[0, 0])
+
+
 def pin_empty(attn):
     """No queries (or a zero batch) gives empty outputs and no error (oxios returns an
     empty result for empty input)."""

@@ -38,6 +38,12 @@ MUTANTS = {
                              "load_elem(J->q, J->dtype, ((b * J->Hq + hq) * Nq + (j < Nq ? j : 0)) * d + c);"),
     "last_key_dropped": ("for (int64_t j = 0; j < N; ++j) {\n    double p", "for (int64_t j = 0; j + 1 < N; ++j) {\n    double p"),
     "sum_without_first_key": ("    l += p;", "    if (j) l += p;"),
+    "sinks_ignored": (" && j >= J->n_sink) sj", ") sj"),
+    "sinks_off_by_one": ("j >= J->n_sink", "j > J->n_sink"),
+    "sinks_override_causal": ("if (J->causal && j > pos)", "if (J->causal && j > pos && j >= J->n_sink)"),
+    "sinks_without_window": ("if (J->window > 0 && pos - j >= J->window && j >= J->n_sink)",
+                             "if ((J->window > 0 && pos - j >= J->window) || (J->n_sink > 0 && j >= J->n_sink))"),
+    "cross_top_left_causal": ("const int64_t pos = i + (N - Nq);", "const int64_t pos = i;"),
 }
 
 
