@@ -82,7 +82,23 @@ def load_traffic(workload: str):
     return rec.get("dram_bytes_per_launch")
 
 
+def kept_keys_per_row(w, i):
+    """Keys each query row i (numpy array) keeps: positions p = i + N - Nq, keys up to p
+    (causal), the window's most recent ones plus the sinks below it."""
+    pos = i + (w.N - w.Nq)
+    hi = np.minimum(pos, w.N - 1) if w.causal else np.full_like(i, w.N - 1)
+    lo = np.maximum(0, pos - w.window + 1) if w.window > 0 else np.zeros_like(i)
+    n = np.maximum(0, hi - lo + 1)
+    if w.window > 0 and w.n_sink > 0:
+        n = n + np.maximum(0, np.minimum(np.minimum(w.n_sink, lo), hi + 1))
+    return n
+
+
 def closed_flops(w) -> float:
+    """The convention for the self-attention workloads; 4 d per kept pair for the
+    general ones (different query and key lengths, sinks)."""
+    if w.nq > 0 or w.n_sink > 0:
+        return float(4.0 * w.d * w.B * w.Hq * kept_keys_per_row(w, np.arange(w.Nq, dtype=np.int64)).sum())
     if w.window > 0:
         return 4.0 * w.B * w.Hq * w.d * (w.N * w.window - w.window * w.window / 2.0)
     f = 4.0 * w.B * w.Hq * w.N * w.N * w.d
@@ -142,17 +158,14 @@ def oracle_sample_rows(w, n_rows: int, offset: int = 0):
     """``n_rows`` flat row indices spread evenly over all heads and query positions (so the
     causal / window work per row averages like the full workload), rotated by
     ``offset``."""
-    total = w.B * w.Hq * w.N
+    total = w.B * w.Hq * w.Nq
     stride = max(1, total // max(1, n_rows))
     start = (offset * 7919) % stride
     return np.arange(start, total, stride, dtype=np.int64)[:n_rows]
 
 
 def rows_flops(w, rows) -> float:
-    i = rows % w.N
-    lo = np.maximum(0, i - w.window + 1) if w.window > 0 else np.zeros_like(i)
-    hi = i if w.causal else np.full_like(i, w.N - 1)
-    return float(4.0 * w.d * np.maximum(0, hi - lo + 1).sum())
+    return float(4.0 * w.d * kept_keys_per_row(w, rows % w.Nq).sum())
 
 
 def time_oracle(w, inputs, seconds: float, offset: int = 0):
@@ -163,12 +176,12 @@ def time_oracle(w, inputs, seconds: float, offset: int = 0):
     threads = oracle.host_threads()
     probe = oracle_sample_rows(w, 64 * threads, offset)
     t0 = time.perf_counter()
-    oracle.attention(q, k, v, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, rows=probe)
+    oracle.attention(q, k, v, scale=w.scale, causal=w.causal, window=w.window, n_sink=w.n_sink, softcap=w.softcap, rows=probe)
     dt = max(time.perf_counter() - t0, 1e-3)
-    n = int(max(threads, min(w.B * w.Hq * w.N, len(probe) * seconds / dt)))
+    n = int(max(threads, min(w.B * w.Hq * w.Nq, len(probe) * seconds / dt)))
     rows = oracle_sample_rows(w, n, offset)
     t0 = time.perf_counter()
-    oracle.attention(q, k, v, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, rows=rows)
+    oracle.attention(q, k, v, scale=w.scale, causal=w.causal, window=w.window, n_sink=w.n_sink, softcap=w.softcap, rows=rows)
     dt = time.perf_counter() - t0
     return rows_flops(w, rows) / dt / 1e12, dt, len(rows), threads
 
@@ -219,7 +232,7 @@ def reference_arm(args, w):
     # per step: a row sample sized for `budget` seconds of oracle work
     probe = oracle_sample_rows(w, 32 * threads)
     t0 = time.perf_counter()
-    oracle.attention(*inputs, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, rows=probe)
+    oracle.attention(*inputs, scale=w.scale, causal=w.causal, window=w.window, n_sink=w.n_sink, softcap=w.softcap, rows=probe)
     dt = max(time.perf_counter() - t0, 1e-3)
     n_rows = int(max(threads, len(probe) * budget / dt))
     total_flop = 0.0
@@ -227,7 +240,7 @@ def reference_arm(args, w):
     for step in range(args.warmup + args.steps):
         rows = oracle_sample_rows(w, n_rows, step)
         t0 = time.perf_counter()
-        oracle.attention(*inputs, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, rows=rows)
+        oracle.attention(*inputs, scale=w.scale, causal=w.causal, window=w.window, n_sink=w.n_sink, softcap=w.softcap, rows=rows)
         dt = time.perf_counter() - t0
         if step >= args.warmup:
             total_flop += rows_flops(w, rows)
@@ -271,11 +284,31 @@ def gpu_arm(args, w):
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
 
-    def step():
-        rc = fa.fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.Hq, w.Hkv,
-                        w.N, w.d, w.scale, w.causal, w.window, w.softcap, sh, w.dtype)
-        if rc != 0:
-            raise fa.FAError(rc, fa.load(), "fa_fwd")
+    general = args.splits > 0 or w.nq > 0 or w.n_sink > 0
+    workspace = None
+    if general:
+        # general entry point (split-KV, cross lengths, sinks); the workspace is
+        # allocated once, outside the timed region
+        ws_bytes = fa.splitkv_workspace_bytes(w.B, w.Hq, w.Nq, w.d, args.splits) if args.splits > 0 else 0
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        ws_ptr = workspace.data_ptr() if args.splits > 0 else None
+        lib = fa.load()
+
+        def launch(qq, kk, vv, oo, ll):
+            rc = lib.fa_fwd_ext(qq.data_ptr(), kk.data_ptr(), vv.data_ptr(), oo.data_ptr(), ll.data_ptr(), w.B, w.Hq,
+                                w.Hkv, w.Nq, w.N, w.d, w.scale, int(w.causal), w.window, w.n_sink, w.softcap,
+                                args.splits, ws_ptr, ws_bytes, sh)
+            if rc != 0:
+                raise fa.FAError(rc, lib, "fa_fwd_ext")
+
+        def step():
+            launch(q, k, v, o, lse)
+    else:
+        def step():
+            rc = fa.fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.Hq, w.Hkv,
+                            w.N, w.d, w.scale, w.causal, w.window, w.softcap, sh, w.dtype)
+            if rc != 0:
+                raise fa.FAError(rc, fa.load(), "fa_fwd")
 
     for _ in range(args.warmup):
         step()
@@ -320,8 +353,11 @@ def gpu_arm(args, w):
             qd.copy_(qp, non_blocking=True)
             kd.copy_(kp, non_blocking=True)
             vd.copy_(vp, non_blocking=True)
-            fa.forward(qd, kd, vd, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, out=o,
-                       lse=lse, stream=stream)
+            if general:
+                launch(qd, kd, vd, o, lse)
+            else:
+                fa.forward(qd, kd, vd, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, out=o,
+                           lse=lse, stream=stream)
             op.copy_(o, non_blocking=True)
             lp.copy_(lse, non_blocking=True)
 
@@ -354,22 +390,37 @@ def gpu_arm(args, w):
 
     peaks, peaks_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    achieved = flop_per_step / (per_launch_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-                "traffic": load_traffic(w.name), "peak_source": f"bf16_tflops (burst) of {peaks_src}",
-                "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
-                "kernel": f"fa_fwd_tc_kernel<{w.d}>", "algorithmic_flop_per_launch": flop_per_step}
+    peak_bw = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    kernel = f"fa_fwd_tc_kernel<{w.d}, {'true' if args.splits > 0 else 'false'}>"
+    # algorithmic bytes: Q, K, V read once, O and LSE written once
+    alg_bytes = float(q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size()
+                      + o.numel() * o.element_size() + lse.numel() * lse.element_size())
+    if flop_per_step / alg_bytes >= peak * 1e12 / (peak_bw * 1e9):
+        achieved = flop_per_step / (per_launch_ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                    "traffic": load_traffic(w.name), "peak_source": f"bf16_tflops (burst) of {peaks_src}",
+                    "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                    "kernel": kernel, "algorithmic_flop_per_launch": flop_per_step}
+    else:  # below the ridge point (one query row per head): bound by reading K and V
+        achieved = alg_bytes / (per_launch_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
+                    "frac": achieved / peak_bw, "traffic": load_traffic(w.name),
+                    "peak_source": f"hbm_gbs of {peaks_src}", "kernel": kernel,
+                    "algorithmic_bytes_per_launch": alg_bytes}
 
     if rank == 0:
         cfg = {"workload": w.name, **{k: v for k, v in w.describe().items() if k != "workload"},
-               "flop_convention": "4 B Hq N^2 d, /2 causal; 4 B Hq d (N W - W^2/2) with a window",
+               "flop_convention": ("4 d per kept (query, key) pair" if (w.nq > 0 or w.n_sink > 0) else
+                                   "4 B Hq N^2 d, /2 causal; 4 B Hq d (N W - W^2/2) with a window"),
                "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{ws} (independent batches)"}
+        if args.splits > 0:
+            cfg["split_kv"] = args.splits
         emit({
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * (2 if args.splits > 0 else 1),
         })
     if ws > 1:
         dist.barrier()
@@ -383,17 +434,19 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.ALL_WORKLOADS))
     ap.add_argument("--batch", type=int, default=None, help="override B (profiling on a smaller case)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=150.0,
                     help="total oracle time budget of the reference arm")
+    ap.add_argument("--splits", type=int, default=0,
+                    help="time the split-KV path with this many key chunks (0: the plain forward)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     args = ap.parse_args(argv)
-    w = workloads.WORKLOADS[args.workload]
+    w = workloads.ALL_WORKLOADS[args.workload]
     if w.dtype != "bfloat16" and args.impl == "ours":
         ap.error("the benchmark times the bf16 tensor-core path")
     if args.batch is not None:

@@ -58,7 +58,8 @@ extern "C" {
 #define FA_ERR_UNSUPPORTED (-3) /* head dim / mask combination this path does not cover,
                                    or the current device is not sm_100                  */
 #define FA_ERR_ALIGN (-4)       /* a pointer breaks the alignment rule above             */
-#define FA_ERR_BAD_ARG (-5)     /* scale not finite or <= 0, softcap not finite          */
+#define FA_ERR_BAD_ARG (-5)     /* scale not finite or <= 0, softcap not finite, n_sink < 0,
+                                   num_splits out of range                               */
 #define FA_ERR_CUDA (-6)        /* a CUDA runtime/driver call failed: fa_last_cuda_error */
 #define FA_ERR_TIMEOUT (-7)     /* a device-side wait exceeded its limit (see below)     */
 #define FA_ERR_WORKSPACE (-8)   /* split-KV workspace NULL, not 16-byte aligned or too small */
@@ -108,6 +109,32 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                    int N, int d, float scale, int causal, int window, float softcap, int num_splits,
                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_fwd_ext -- the general form: queries and keys of different lengths (cross-attention,
+ * decoding against a key/value cache), attention sinks, and optional split-KV.
+ *   q, o : [B, Hq, Nq, d];  k, v : [B, Hkv, Nk, d];  lse : [B, Hq, Nq].
+ *   Nq, Nk : query rows and key rows per head (>= 0).  Query row i sits at position
+ *            p = i + (Nk - Nq) of the key sequence: the queries are the last Nq
+ *            positions (with Nq == Nk this is self-attention, p = i).  The causal and
+ *            window masks use p: keys j > p are masked (causal), and keys with
+ *            p - j >= window (window > 0).  A row with no valid key (Nq > Nk, causal,
+ *            rows i < Nq - Nk; or Nk == 0) gets O = 0 and LSE = -inf.
+ *            Cross-attention: oxios flash_attention.rs, FlashAttention::cross_attention
+ *            (queries from one sequence, keys and values from another).
+ *   n_sink : >= 0.  With a window, keys 0 .. n_sink-1 (the attention sinks) are exempt
+ *            from the window; they stay under the causal mask.  "Module 16: Efficient and
+ *            Long Attention", section 16.6, keeps the first 4 tokens beside the sliding
+ *            window.  Without a window every key is kept anyway and n_sink has no effect.
+ *   num_splits : 0 runs the plain forward (workspace may be NULL); 1 .. FA_MAX_SPLITS runs
+ *            split-KV as fa_fwd_splitkv with a workspace of at least
+ *            fa_fwd_splitkv_workspace(B, Hq, Nq, d, num_splits) bytes.
+ *   Other arguments, precision and errors as fa_fwd and fa_fwd_splitkv; k and v may be
+ *   NULL when Nk == 0.  FA_ERR_BAD_ARG for n_sink < 0 or num_splits out of range.
+ */
+int fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+               int Nk, int d, float scale, int causal, int window, int n_sink, float softcap, int num_splits,
+               void* workspace, size_t workspace_bytes, void* stream);
 
 /* fa_fwd_splitkv_workspace -- bytes of workspace fa_fwd_splitkv needs (0 for an empty or
  * invalid problem): num_splits * B * Hq * N * (d + 1) * 4. */

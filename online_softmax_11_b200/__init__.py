@@ -36,7 +36,7 @@ ERRORS = {
 STATIC_SCRATCH_BYTES = 32 << 20
 MAX_SPLITS = 64
 # every symbol include/fa.h declares
-EXPORTS = ["fa_fwd", "fa_fwd_f32", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace", "fa_fwd_splitkv_static",
+EXPORTS = ["fa_fwd", "fa_fwd_f32", "fa_fwd_ext", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace", "fa_fwd_splitkv_static",
            "fa_check_status", "fa_selftest_wait_timeout", "fa_strerror", "fa_last_cuda_error", "fa_version"]
 
 _lock = threading.Lock()
@@ -76,6 +76,8 @@ def load():
         lib.fa_fwd_splitkv.argtypes = sig[:-1] + [i, vp, ctypes.c_size_t, vp]
         lib.fa_fwd_splitkv_static.restype = i
         lib.fa_fwd_splitkv_static.argtypes = sig[:-1] + [i, vp]
+        lib.fa_fwd_ext.restype = i
+        lib.fa_fwd_ext.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, f, i, vp, ctypes.c_size_t, vp]
         lib.fa_fwd_splitkv_workspace.restype = ctypes.c_size_t
         lib.fa_fwd_splitkv_workspace.argtypes = [i, i, i, i, i]
         lib.fa_check_status.restype = i
@@ -183,6 +185,45 @@ def forward_splitkv(q, k, v, *, num_splits: int, scale: float | None = None, cau
     return out, lse
 
 
+def forward_ext(q, k, v, *, scale: float | None = None, causal: bool = False, window: int = 0, n_sink: int = 0,
+                softcap: float = 0.0, num_splits: int = 0, out=None, lse=None, workspace=None, stream=None):
+    """General bf16 forward through ``fa_fwd_ext``: q [B, Hq, Nq, d] against k, v
+    [B, Hkv, Nk, d] (queries at the last Nq key positions), attention sinks beside a
+    window, and split-KV when ``num_splits`` >= 1 (workspace allocated here with torch
+    when not given)."""
+    import torch
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, N, d]")
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("fa_fwd_ext takes bfloat16 q, k, v")
+    if k.shape != (B, Hkv, Nk, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, Nk, d] with q's B and d")
+    for t in (q, k, v):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    if scale is None:
+        scale = float(torch.tensor(1.0, dtype=torch.float32) / torch.sqrt(torch.tensor(float(d), dtype=torch.float32)))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    ws_ptr, ws_bytes = None, 0
+    if num_splits > 0:
+        if workspace is None:
+            need = splitkv_workspace_bytes(B, Hq, Nq, d, num_splits)
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        rc = load().fa_fwd_ext(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
+                               Nq, Nk, d, float(scale), int(bool(causal)), int(window), int(n_sink), float(softcap),
+                               int(num_splits), ws_ptr, ws_bytes, _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, load(), "fa_fwd_ext")
+    return out, lse
+
+
 def check_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return load().fa_check_status(_stream_handle(stream))
@@ -204,5 +245,5 @@ def attention_flops(B: int, Hq: int, N: int, d: int, causal: bool = False, windo
     return 4.0 * d * B * Hq * pairs
 
 
-__all__ = ["forward", "forward_splitkv", "splitkv_workspace_bytes", "fwd_raw", "load", "check_status",
+__all__ = ["forward", "forward_ext", "forward_splitkv", "splitkv_workspace_bytes", "fwd_raw", "load", "check_status",
            "selftest_wait_timeout", "attention_flops", "FAError", "EXPORTS", "LIB_PATH", "MAX_SPLITS"]

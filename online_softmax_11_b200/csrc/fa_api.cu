@@ -121,19 +121,22 @@ int make_map(CUtensorMap* map, const void* base, int heads, int N, int d) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// Checks shared by both entry points.  Returns FA_OK, an error, or 1 for "empty problem".
-int check_common(const void* q, const void* k, const void* v, const void* o, int B, int Hq, int Hkv, int N, int d,
-                 float scale, int causal, int window, float softcap) {
-  if (B < 0 || Hq < 0 || Hkv < 0 || N < 0 || d < 0) return FA_ERR_BAD_SHAPE;
+// Checks shared by every entry point.  Returns FA_OK, an error, or 1 for "empty problem"
+// (no query rows).  With query rows but no keys (Nk == 0) k and v may be NULL.
+int check_common(const void* q, const void* k, const void* v, const void* o, int B, int Hq, int Hkv, int Nq, int Nk,
+                 int d, float scale, int causal, int window, int n_sink, float softcap) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0 || d < 0) return FA_ERR_BAD_SHAPE;
   if (Hkv == 0 || (Hq % Hkv) != 0) return FA_ERR_BAD_SHAPE;
-  if (!std::isfinite(scale) || !(scale > 0.f) || !std::isfinite(softcap)) return FA_ERR_BAD_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f) || !std::isfinite(softcap) || n_sink < 0) return FA_ERR_BAD_ARG;
   if (window > 0 && !causal) return FA_ERR_UNSUPPORTED;
   // element counts must fit the kernels' index arithmetic
-  const long long rows = static_cast<long long>(B) * Hq * N;
-  if (rows > (1ll << 31) - 1 || static_cast<long long>(B) * Hq > (1ll << 31) - 1) return FA_ERR_BAD_SHAPE;
-  if (B == 0 || Hq == 0 || N == 0) return 1;
+  const long long rows = static_cast<long long>(B) * Hq * Nq;
+  const long long kv_rows = static_cast<long long>(B) * Hkv * Nk;
+  if (rows > (1ll << 31) - 1 || kv_rows > (1ll << 31) - 1 || static_cast<long long>(B) * Hq > (1ll << 31) - 1)
+    return FA_ERR_BAD_SHAPE;
+  if (B == 0 || Hq == 0 || Nq == 0) return 1;
   if (d == 0) return FA_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !o) return FA_ERR_NULL_PTR;
+  if (!q || !o || (Nk > 0 && (!k || !v))) return FA_ERR_NULL_PTR;
   return FA_OK;
 }
 
@@ -166,20 +169,34 @@ const char* fa_strerror(int code) {
 
 namespace {
 
+// O = 0 and LSE = -inf for every row: the merge of zero chunks (query rows, no keys).
+int launch_no_keys(void* o, float* lse, long long rows, int d, cudaStream_t s) {
+  const unsigned mgrid = static_cast<unsigned>((rows + fa::kMergeRowsPerBlock - 1) / fa::kMergeRowsPerBlock);
+  if (d == 128)
+    fa::fa_merge_splits_kernel<128><<<mgrid, 32 * fa::kMergeRowsPerBlock, 0, s>>>(
+        nullptr, nullptr, static_cast<__nv_bfloat16*>(o), lse, rows, 0);
+  else
+    fa::fa_merge_splits_kernel<64><<<mgrid, 32 * fa::kMergeRowsPerBlock, 0, s>>>(
+        nullptr, nullptr, static_cast<__nv_bfloat16*>(o), lse, rows, 0);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
 // Launch the tensor-core kernel: plain (num_splits == 0: bf16 O and fp32 LSE) or split-KV
 // (num_splits >= 1: fp32 partials into o_part / lse_part, then the merge kernel).
-int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
-              int d, float scale, int causal, int window, float softcap, int num_splits, float* o_part,
-              float* lse_part, cudaStream_t s) {
+int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+              int Nk, int d, float scale, int causal, int window, int n_sink, float softcap, int num_splits,
+              float* o_part, float* lse_part, cudaStream_t s) {
   int rc;
   int dev, num_sms = 0;
   if ((rc = current_device(&dev)) != FA_OK) return rc;
   if ((rc = prepare_device(dev, &num_sms)) != FA_OK) return rc;
+  if (Nk == 0) return launch_no_keys(o, lse, static_cast<long long>(B) * Hq * Nq, d, s);
 
   CUtensorMap mq, mk, mv;
-  if ((rc = make_map(&mq, q, B * Hq, N, d)) != FA_OK) return rc;
-  if ((rc = make_map(&mk, k, B * Hkv, N, d)) != FA_OK) return rc;
-  if ((rc = make_map(&mv, v, B * Hkv, N, d)) != FA_OK) return rc;
+  if ((rc = make_map(&mq, q, B * Hq, Nq, d)) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * Hkv, Nk, d)) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * Hkv, Nk, d)) != FA_OK) return rc;
 
   namespace tc = fa::tc;
   const bool split = num_splits >= 1;
@@ -188,9 +205,12 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.lse = lse;
   p.Hq = Hq;
   p.Hkv = Hkv;
-  p.N = N;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.pos_off = Nk - Nq;
+  p.n_sink = window > 0 ? n_sink : 0;  // sinks only matter beside a window
   p.n_bh = B * Hq;
-  p.n_qp = (N + tc::NQ * tc::BM - 1) / (tc::NQ * tc::BM);
+  p.n_qp = (Nq + tc::NQ * tc::BM - 1) / (tc::NQ * tc::BM);
   p.units_per_head = (p.n_qp + 1) / 2;
   p.causal = causal ? 1 : 0;
   p.window = window > 0 ? window : 0;
@@ -225,7 +245,7 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   if (split) {
-    const long long rows = static_cast<long long>(B) * Hq * N;
+    const long long rows = static_cast<long long>(B) * Hq * Nq;
     const unsigned mgrid = static_cast<unsigned>((rows + fa::kMergeRowsPerBlock - 1) / fa::kMergeRowsPerBlock);
     if (d == 128)
       fa::fa_merge_splits_kernel<128><<<mgrid, 32 * fa::kMergeRowsPerBlock, 0, s>>>(
@@ -240,8 +260,8 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
 }
 
 int check_bf16(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int Hq, int Hkv,
-               int N, int d, float scale, int causal, int window, float softcap) {
-  int rc = check_common(q, k, v, o, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+               int Nq, int Nk, int d, float scale, int causal, int window, int n_sink, float softcap) {
+  int rc = check_common(q, k, v, o, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, n_sink, softcap);
   if (rc != FA_OK) return rc;  // 1 = empty problem
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4)))
@@ -255,10 +275,10 @@ extern "C" {
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d,
            float scale, int causal, int window, float softcap, void* stream) {
-  int rc = check_bf16(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+  int rc = check_bf16(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, causal, window, 0, softcap);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
-  return launch_tc(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap, 0, nullptr, nullptr,
+  return launch_tc(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, causal, window, 0, softcap, 0, nullptr, nullptr,
                    static_cast<cudaStream_t>(stream));
 }
 
@@ -271,22 +291,36 @@ size_t fa_fwd_splitkv_workspace(int B, int Hq, int N, int d, int num_splits) {
 int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
                    int d, float scale, int causal, int window, float softcap, int num_splits, void* workspace,
                    size_t workspace_bytes, void* stream) {
-  int rc = check_bf16(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+  const int rc = check_bf16(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, causal, window, 0, softcap);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
-  if (num_splits < 1 || num_splits > FA_MAX_SPLITS) return FA_ERR_BAD_ARG;
-  const size_t need = fa_fwd_splitkv_workspace(B, Hq, N, d, num_splits);
+  if (num_splits < 1 || num_splits > FA_MAX_SPLITS) return FA_ERR_BAD_ARG;  // 0 means "no split" only in fa_fwd_ext
+  return fa_fwd_ext(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, causal, window, 0, softcap, num_splits, workspace,
+                    workspace_bytes, stream);
+}
+
+int fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+               int Nk, int d, float scale, int causal, int window, int n_sink, float softcap, int num_splits,
+               void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_bf16(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, n_sink, softcap);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (num_splits < 0 || num_splits > FA_MAX_SPLITS) return FA_ERR_BAD_ARG;
+  if (num_splits == 0)
+    return launch_tc(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, n_sink, softcap, 0, nullptr,
+                     nullptr, static_cast<cudaStream_t>(stream));
+  const size_t need = fa_fwd_splitkv_workspace(B, Hq, Nq, d, num_splits);
   if (workspace == nullptr || !aligned(workspace, 16) || workspace_bytes < need) return FA_ERR_WORKSPACE;
-  const size_t rows = static_cast<size_t>(B) * Hq * N;
+  const size_t rows = static_cast<size_t>(B) * Hq * Nq;
   float* o_part = static_cast<float*>(workspace);
   float* lse_part = o_part + static_cast<size_t>(num_splits) * rows * d;
-  return launch_tc(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap, num_splits, o_part, lse_part,
-                   static_cast<cudaStream_t>(stream));
+  return launch_tc(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, n_sink, softcap, num_splits, o_part,
+                   lse_part, static_cast<cudaStream_t>(stream));
 }
 
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Hq, int Hkv, int N,
                int d, float scale, int causal, int window, float softcap, void* stream) {
-  int rc = check_common(q, k, v, o, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+  int rc = check_common(q, k, v, o, B, Hq, Hkv, N, N, d, scale, causal, window, 0, softcap);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
   if (d < 1 || d > fa::f32path::kMaxD) return FA_ERR_UNSUPPORTED;
@@ -361,7 +395,7 @@ extern "C" {
 int fa_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                           int N, int d, float scale, int causal, int window, float softcap, int num_splits,
                           void* stream) {
-  int rc = check_bf16(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap);
+  int rc = check_bf16(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, causal, window, 0, softcap);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
   if (num_splits < 1 || num_splits > FA_MAX_SPLITS) return FA_ERR_BAD_ARG;
@@ -376,8 +410,8 @@ int fa_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, 
   const size_t rows = static_cast<size_t>(B) * Hq * N;
   float* o_part = static_cast<float*>(scratch);
   float* lse_part = o_part + static_cast<size_t>(num_splits) * rows * d;
-  return launch_tc(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, window, softcap, num_splits, o_part, lse_part,
-                   static_cast<cudaStream_t>(stream));
+  return launch_tc(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, causal, window, 0, softcap, num_splits, o_part,
+                   lse_part, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

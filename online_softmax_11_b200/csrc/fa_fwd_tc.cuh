@@ -105,9 +105,12 @@ struct Layout {
 struct Params {
   __nv_bfloat16* o;
   float* lse;
-  int Hq, Hkv, N;
+  int Hq, Hkv;
+  int Nq, Nk;          // query rows and key rows per head
+  int pos_off;         // Nk - Nq: query row i sits at position i + pos_off of the keys
+  int n_sink;          // keys [0, n_sink) are exempt from the window (0: none)
   int n_bh;            // B * Hq
-  int n_qp;            // ceil(N / 256): query-tile pairs per head
+  int n_qp;            // ceil(Nq / 256): query-tile pairs per head
   int units_per_head;  // ceil(n_qp / 2)
   int n_units;         // n_bh * units_per_head
   int causal;
@@ -121,8 +124,8 @@ struct Params {
   // chunks, each chunk a work tile of its own, writing a partial O (fp32, normalised
   // within the chunk) and a partial LSE for a merge pass (fa_merge.cuh)
   int num_splits;      // 1: plain forward, outputs o / lse
-  float* o_part;       // [num_splits][B*Hq][N][d]
-  float* lse_part;     // [num_splits][B*Hq][N]
+  float* o_part;       // [num_splits][B*Hq][Nq][d]
+  float* lse_part;     // [num_splits][B*Hq][Nq]
 };
 
 // Accurate tanh for the soft-cap: Taylor series about 0 through x^11 for |x| < 0.3
@@ -239,58 +242,94 @@ __device__ __forceinline__ float make_p(const float (&s)[kHalf], uint32_t taddr_
   return lsum.x + lsum.y;
 }
 
-// 64 scores of the row (tile columns c0 .. c0+63) from TMEM, masked to the row's valid
-// column range [c_lo, c_hi] when the tile needs a mask (-inf outside).
-__device__ __forceinline__ void load_half(uint32_t taddr, int c0, bool need_mask, int c_lo, int c_hi,
+// 64 scores of the row (tile columns c0 .. c0+63) from TMEM, masked when the tile needs a
+// mask: -inf above column c_hi and in the hole [h_lo, h_hi) (the columns below the window
+// that are not attention sinks; h_lo = 0 without sinks).
+__device__ __forceinline__ void load_half(uint32_t taddr, int c0, bool need_mask, int h_lo, int h_hi, int c_hi,
                                           float (&s)[kHalf]) {
   uint32_t r[kHalf];
   tmem_ld64_wait(taddr, r);
 #pragma unroll
   for (int c = 0; c < kHalf; ++c) s[c] = __uint_as_float(r[c]);
   if (need_mask) {
+    const uint32_t hole = static_cast<uint32_t>(h_hi - h_lo);
 #pragma unroll
-    for (int c = 0; c < kHalf; ++c) s[c] = (c0 + c < c_lo || c0 + c > c_hi) ? -CUDART_INF_F : s[c];
+    for (int c = 0; c < kHalf; ++c)
+      s[c] = (static_cast<uint32_t>(c0 + c - h_lo) < hole || c0 + c > c_hi) ? -CUDART_INF_F : s[c];
   }
 }
 
-// Key-tile range of one query tile: [lo, hi) of 128-key tiles.
-struct TileRange {
-  int r0, r1;  // first / last query row (r1 < N)
-  int lo, hi;
-  bool active;  // the tile has rows below N
-  bool part;    // ... and key tiles to process in this work tile (lo < hi)
+// A set of 128-key tiles as two ascending runs, [a0, a1) then [b0, b1) with a1 <= b0.
+// The first run holds attention-sink tiles when they are apart from the window's tiles;
+// otherwise it is empty and everything is in the second run.  Empty runs are (0, 0).
+struct TileSet {
+  int a0, a1, b0, b1;
+  __device__ int count() const { return (a1 - a0) + (b1 - b0); }
+  __device__ int at(int n) const { return n < a1 - a0 ? a0 + n : b0 + (n - (a1 - a0)); }
+  __device__ bool has(int j) const { return (j >= a0 && j < a1) || (j >= b0 && j < b1); }
+  __device__ int first() const { return a1 > a0 ? a0 : b0; }
+  __device__ int last() const { return b1 > b0 ? b1 - 1 : a1 - 1; }
 };
 
-__device__ __forceinline__ TileRange tile_range(int r0, int N, int nkv, int causal, int window) {
-  TileRange t;
-  t.r0 = r0;
-  t.active = r0 < N;
-  t.r1 = min(N, r0 + BM) - 1;
-  t.lo = 0;
-  t.hi = nkv;
-  if (causal) t.hi = min(nkv, t.r1 / BN + 1);
-  if (window > 0) t.lo = max(0, t.r0 - window + 1) / BN;
-  if (!t.active) t.lo = t.hi = 0;
-  t.part = t.active && t.lo < t.hi;
-  return t;
+__device__ __forceinline__ void run_and(int x0, int x1, int y0, int y1, int& r0, int& r1) {
+  r0 = max(x0, y0);
+  r1 = min(x1, y1);
+  if (r1 <= r0) r0 = r1 = 0;
 }
 
-__device__ __forceinline__ bool participates(const TileRange& t, int j) { return t.active && j >= t.lo && j < t.hi; }
+// Key tiles of one query tile: rows r0 .. r1 (r1 < Nq) at positions r + pos_off.
+struct TileRange {
+  int r0, r1;   // first / last query row
+  TileSet ks;   // key tiles this work tile streams for it
+  bool active;  // the tile has rows below Nq
+  bool part;    // ... and key tiles to process in this work tile
+};
+
+__device__ __forceinline__ TileRange tile_range(const Params& p, int r0, int nkv) {
+  TileRange t;
+  t.r0 = r0;
+  t.active = r0 < p.Nq;
+  t.r1 = min(p.Nq, r0 + BM) - 1;
+  const int pr0 = r0 + p.pos_off, pr1 = t.r1 + p.pos_off;
+  int lo = 0, hi = nkv;
+  if (p.causal) hi = pr1 < 0 ? 0 : min(nkv, pr1 / BN + 1);
+  if (p.window > 0) lo = min(hi, max(0, pr0 - p.window + 1) / BN);
+  t.ks = TileSet{0, 0, lo, hi};
+  if (p.window > 0 && p.n_sink > 0) {
+    const int sink_tiles = min(hi, (p.n_sink + BN - 1) / BN);
+    if (lo <= sink_tiles) t.ks.b0 = 0;  // sinks and window join up: one run from key 0
+    else t.ks.a1 = sink_tiles;
+  }
+  if (!t.active || t.ks.count() <= 0) t.ks = TileSet{0, 0, 0, 0};
+  t.part = t.ks.count() > 0;
+  return t;
+}
 
 // One work tile: (batch*head, query-tile pair, key chunk) and the key tiles it streams.
 struct WorkTile {
   int bh, kvh;
   int split;   // key chunk (0 without split-KV)
   TileRange tr0, tr1;
-  int lo, hi;  // union key-tile range of the participating query tiles
+  TileSet ks;  // key tiles streamed: the union of both query tiles' sets (or a chunk of it)
   __device__ const TileRange& tr(int i) const { return i == 0 ? tr0 : tr1; }
 };
 
-__device__ __forceinline__ void clip(TileRange& t, int jlo, int jhi) {
-  t.lo = max(t.lo, jlo);
-  t.hi = min(t.hi, jhi);
-  t.part = t.active && t.lo < t.hi;
-  if (!t.part) t.lo = t.hi = 0;
+// Keep the part of t's tiles inside chunk c.  Each run of t meets at most one run of c
+// (sink tiles lie below every window tile of the pair when the union keeps them apart).
+__device__ __forceinline__ void clip(TileRange& t, const TileSet& c) {
+  int x0, x1, y0, y1;
+  TileSet k;
+  run_and(t.ks.a0, t.ks.a1, c.a0, c.a1, x0, x1);
+  run_and(t.ks.a0, t.ks.a1, c.b0, c.b1, y0, y1);
+  k.a0 = x1 > x0 ? x0 : y0;
+  k.a1 = x1 > x0 ? x1 : y1;
+  run_and(t.ks.b0, t.ks.b1, c.a0, c.a1, x0, x1);
+  run_and(t.ks.b0, t.ks.b1, c.b0, c.b1, y0, y1);
+  k.b0 = x1 > x0 ? x0 : y0;
+  k.b1 = x1 > x0 ? x1 : y1;
+  t.ks = k;
+  t.part = t.active && k.count() > 0;
+  if (!t.part) t.ks = TileSet{0, 0, 0, 0};
 }
 
 __device__ __forceinline__ WorkTile make_work_tile(const Params& p, int bh, int qp, int split) {
@@ -300,29 +339,42 @@ __device__ __forceinline__ WorkTile make_work_tile(const Params& p, int bh, int 
   const int b = bh / p.Hq;
   const int hq = bh - b * p.Hq;
   w.kvh = b * p.Hkv + hq / (p.Hq / p.Hkv);
-  const int nkv = (p.N + BN - 1) / BN;
-  w.tr0 = tile_range(qp * NQ * BM, p.N, nkv, p.causal, p.window);
-  w.tr1 = tile_range(qp * NQ * BM + BM, p.N, nkv, p.causal, p.window);
-  int ulo = w.tr0.lo, uhi = w.tr0.hi;
-  if (w.tr1.active) {
-    ulo = min(ulo, w.tr1.lo);
-    uhi = max(uhi, w.tr1.hi);
+  const int nkv = (p.Nk + BN - 1) / BN;
+  w.tr0 = tile_range(p, qp * NQ * BM, nkv);
+  w.tr1 = tile_range(p, qp * NQ * BM + BM, nkv);
+  // union: sink runs start at tile 0; the window runs of the two query tiles overlap or
+  // touch (the second starts at most one tile past the first's end), so the union is
+  // again two runs, joined when the sink run reaches the window run
+  const TileSet& s0 = w.tr0.ks;
+  const TileSet& s1 = w.tr1.ks;
+  TileSet u{0, max(s0.a1, s1.a1), 0, 0};
+  if (s0.b1 > s0.b0 && s1.b1 > s1.b0) {
+    u.b0 = min(s0.b0, s1.b0);
+    u.b1 = max(s0.b1, s1.b1);
+  } else if (s0.b1 > s0.b0) {
+    u.b0 = s0.b0;
+    u.b1 = s0.b1;
+  } else {
+    u.b0 = s1.b0;
+    u.b1 = s1.b1;
   }
+  if (u.a1 > 0 && u.a1 >= u.b0) u = TileSet{0, 0, 0, max(u.a1, u.b1)};
+  w.ks = u;
   if (p.num_splits > 1) {  // this work tile keeps chunk `split` of the pair's key tiles
-    const int T = uhi - ulo;
-    const int jlo = ulo + (split * T) / p.num_splits;
-    const int jhi = ulo + ((split + 1) * T) / p.num_splits;
-    clip(w.tr0, jlo, jhi);
-    clip(w.tr1, jlo, jhi);
-  }
-  w.lo = w.hi = 0;
-  if (w.tr0.part) {
-    w.lo = w.tr0.lo;
-    w.hi = w.tr0.hi;
-  }
-  if (w.tr1.part) {
-    w.lo = w.tr0.part ? min(w.lo, w.tr1.lo) : w.tr1.lo;
-    w.hi = max(w.hi, w.tr1.hi);
+    const int T = u.count();
+    const int c0 = (split * T) / p.num_splits;
+    const int c1 = ((split + 1) * T) / p.num_splits;
+    const int na = u.a1 - u.a0;
+    TileSet c;
+    c.a0 = u.a0 + min(c0, na);
+    c.a1 = u.a0 + min(c1, na);
+    c.b0 = u.b0 + max(c0 - na, 0);
+    c.b1 = u.b0 + max(c1 - na, 0);
+    if (c.a1 <= c.a0) c.a0 = c.a1 = 0;
+    if (c.b1 <= c.b0) c.b0 = c.b1 = 0;
+    clip(w.tr0, c);
+    clip(w.tr1, c);
+    w.ks = c;
   }
   return w;
 }
@@ -417,7 +469,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         w.bh);
           ++q_cnt[i];
         }
-        for (int j = w.lo; j < w.hi; ++j) {
+        const int T = w.ks.count();
+        for (int n = 0; n < T; ++n) {
+          const int j = w.ks.at(n);
           for (int which = 0; which < 2; ++which) {
             const int s = issued % L::kStages;
             const uint32_t fill = issued / L::kStages;
@@ -467,9 +521,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for_each_tile(p, [&](const WorkTile& w) {
         const TileRange& t = w.tr(i);
         uint32_t o_acc = 0;
-        const int T = w.hi - w.lo;
+        const int T = w.ks.count();
+        const int t_first = t.ks.first(), t_last = t.ks.last();
         for (int n = 0; n <= T; ++n) {
-          const int j = w.lo + n;
+          const int j = n < T ? w.ks.at(n) : -1;       // key tile whose S is issued now
+          const int jp = n > 0 ? w.ks.at(n - 1) : -1;  // key tile whose P.V is issued now
           const int kidx = used + 2 * n;
           const int vidx = kidx - 1;
           const int kslot = kidx % L::kStages;
@@ -478,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // proxy on shared memory).  P, written to tensor memory by the softmax warps'
           // tcgen05.st, also needs tcgen05.fence::after_thread_sync after its barrier.
           if (n > 0) {
-            if (participates(t, j - 1)) {
+            if (t.part && t.ks.has(jp)) {
               if (!mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
               if (!mbar_wait(&bars[L::kBarPFull + i], p_phase, ctl)) return false;
               p_phase ^= 1u;
@@ -487,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               // of V (128 B each); the two 64-column slabs of V are kHalfBytes apart
               mma_ts_kloop8(d_o, d_s, dvring + ((vslot * L::kTileBytes) >> 4), kIdescPV, o_acc);
               o_acc = 1;
-              if (!participates(t, j)) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
+              if (jp == t_last) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
               mma_commit(&bars[L::kBarKvEmpty + vslot]);
             } else {
               // not used by this query tile: release it, but only once this fill has
@@ -497,15 +553,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (n < T) {
-            if (participates(t, j)) {
+            if (t.part && t.ks.has(j)) {
               if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
-              if (j == t.lo) {  // first use of this work tile's Q_i
+              if (j == t_first) {  // first use of this work tile's Q_i
                 if (!mbar_wait(&bars[L::kBarQFull + i], q_cnt & 1u, ctl)) return false;
                 ++q_cnt;
               }
               mma_ss_kloop<D / 16>(d_s, dq, dring + ((kslot * L::kTileBytes) >> 4), kIdescS);
               mma_commit(&bars[L::kBarSFull + i]);
-              if (j == t.hi - 1) mma_commit(&bars[L::kBarQEmpty + i]);  // Q_i no longer read
+              if (j == t_last) mma_commit(&bars[L::kBarQEmpty + i]);  // Q_i no longer read
               mma_commit(&bars[L::kBarKvEmpty + kslot]);
             } else {
               if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
@@ -533,27 +589,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for_each_tile(p, [&](const WorkTile& w) {
       const TileRange& t = w.tr(i);
-      if (!t.active) return true;  // rows past N: nothing to write
+      if (!t.active) return true;  // rows past Nq: nothing to write
       const int row = t.r0 + trow;
+      const int pos = row + p.pos_off;  // the row's position in the key sequence
+      const int pr0 = t.r0 + p.pos_off, pr1 = t.r1 + p.pos_off;
       float m = -CUDART_INF_F;  // running reference maximum (log2 units)
       float l = 0.f;            // running sum of P (fp32) relative to m
       float lr = 0.f;           // normaliser of O (l with each tile maximum's P as rounded)
       bool o_valid = false;
 
-      for (int j = t.lo; j < t.hi; ++j) {
+      const int T = t.ks.count();
+      for (int n = 0; n < T; ++n) {
+        const int j = t.ks.at(n);
         // tcgen05.ld/st are warp-collective: the whole warp leaves together or not at all
         if (!__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarSFull + i], s_phase, ctl))) return false;
         s_phase ^= 1u;
         tc_fence_after();
 
         const int k0 = j * BN;
-        const bool need_mask = (k0 + BN > p.N) || (p.causal && k0 + BN - 1 > t.r0) ||
-                               (p.window > 0 && t.r1 - k0 >= p.window);
-        // valid keys of this row form one column range [c_lo, c_hi] of the tile: keys
-        // below N, at most the query's own position (causal), and within the window
-        int c_hi = min(BN - 1, p.N - 1 - k0);
-        if (p.causal) c_hi = min(c_hi, row - k0);
-        const int c_lo = p.window > 0 ? max(0, row - p.window + 1 - k0) : 0;
+        const bool need_mask = (k0 + BN > p.Nk) || (p.causal && k0 + BN - 1 > pr0) ||
+                               (p.window > 0 && pr1 - k0 >= p.window && k0 + BN > p.n_sink);
+        // valid keys of this row: columns up to c_hi (keys below Nk, at most the query's
+        // own position when causal), minus the hole [h_lo, h_hi) of keys that are below
+        // the window and are not attention sinks
+        int c_hi = min(BN - 1, p.Nk - 1 - k0);
+        if (p.causal) c_hi = min(c_hi, pos - k0);
+        const int w_lo = p.window > 0 ? max(0, pos - p.window + 1 - k0) : 0;  // window's first column
+        const int h_lo = min(max(0, p.n_sink - k0), w_lo);
+        const int h_hi = w_lo;
 
         // Pass 1: row maximum (and minimum, for the soft-cap range check) over the two
         // 64-score halves with three-input max: three chains over the columns whose exp2
@@ -565,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float s[kHalf];
-          load_half(lane_base + colS + h * kHalf, h * kHalf, need_mask, c_lo, c_hi, s);
+          load_half(lane_base + colS + h * kHalf, h * kHalf, need_mask, h_lo, h_hi, c_hi, s);
 #pragma unroll
           for (int c = 0; c < kHalf; c += 8) {
             mx0 = fmax3(mx0, s[c], s[c + 1]);
@@ -627,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float s[kHalf];
-          load_half(lane_base + colS + h * kHalf, h * kHalf, need_mask, c_lo, c_hi, s);
+          load_half(lane_base + colS + h * kHalf, h * kHalf, need_mask, h_lo, h_hi, c_hi, s);
           const uint32_t tp = lane_base + colS + h * (kHalf / 2);
           if (!p.use_softcap) {
             if (need_mask)
@@ -676,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float inv = lr > 0.f ? 1.0f / lr : 0.f;
       if constexpr (kSplit) {
-        const int64_t prow = (static_cast<int64_t>(w.split) * p.n_bh + w.bh) * p.N + row;
+        const int64_t prow = (static_cast<int64_t>(w.split) * p.n_bh + w.bh) * p.Nq + row;
         float* orow = p.o_part + prow * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -687,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int x = 0; x < 32; ++x) r[x] = 0u;
           }
-          if (row < p.N) {
+          if (row < p.Nq) {
             float4* dst = reinterpret_cast<float4*>(orow + c * 32);
 #pragma unroll
             for (int x = 0; x < 8; ++x)
@@ -695,15 +758,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    __uint_as_float(r[4 * x + 2]) * inv, __uint_as_float(r[4 * x + 3]) * inv);
           }
         }
-        if (row < p.N) p.lse_part[prow] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+        if (row < p.Nq) p.lse_part[prow] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
         return true;
       }
-      __nv_bfloat16* orow = p.o + (static_cast<int64_t>(w.bh) * p.N + row) * D;
+      __nv_bfloat16* orow = p.o + (static_cast<int64_t>(w.bh) * p.Nq + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32_wait(lane_base + colO + c * 32, r);
-        if (row < p.N) {
+        if (t.part) {
+          tmem_ld32_wait(lane_base + colO + c * 32, r);
+        } else {  // no key at all for this query tile (fewer keys than queries, causal)
+#pragma unroll
+          for (int x = 0; x < 32; ++x) r[x] = 0u;
+        }
+        if (row < p.Nq) {
           uint4 v4[4];
           uint32_t* wp = reinterpret_cast<uint32_t*>(v4);
 #pragma unroll
@@ -714,8 +782,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int x = 0; x < 4; ++x) dst[x] = v4[x];
         }
       }
-      if (p.lse != nullptr && row < p.N)
-        p.lse[static_cast<int64_t>(w.bh) * p.N + row] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+      if (p.lse != nullptr && row < p.Nq)
+        p.lse[static_cast<int64_t>(w.bh) * p.Nq + row] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
       return true;
     });
   }

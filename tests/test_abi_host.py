@@ -133,3 +133,30 @@ def test_splitkv_argument_errors(lib):
     assert call_split(lib, d=32) == -3
     assert call_split(lib, Hq=3) == -2
     assert call_split(lib, q=None, k=None, v=None, o=None, lse=None, ws=None, N=0) == 0  # empty problem
+
+
+def call_ext(lib, num_splits=0, ws=None, ws_bytes=0, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, Nq=8, Nk=8, d=64, scale=0.125, causal=1,
+             window=0, n_sink=0, softcap=0.0)
+    a.update(kw)
+    return lib.fa_fwd_ext(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"],
+                          a["d"], a["scale"], a["causal"], a["window"], a["n_sink"], a["softcap"], num_splits, ws,
+                          ws_bytes, None)
+
+
+def test_ext_argument_errors(lib):
+    assert call_ext(lib, Nq=-1) == -2
+    assert call_ext(lib, Nk=-1) == -2
+    assert call_ext(lib, n_sink=-1) == -5
+    assert call_ext(lib, num_splits=-1) == -5
+    assert call_ext(lib, num_splits=fa.MAX_SPLITS + 1) == -5
+    assert call_ext(lib, num_splits=2) == -8                      # split-KV needs a workspace
+    assert call_ext(lib, num_splits=2, ws=FAKE, ws_bytes=16) == -8
+    assert call_ext(lib, window=4, causal=0) == -3
+    assert call_ext(lib, d=96) == -3
+    assert call_ext(lib, q=None) == -1
+    assert call_ext(lib, k=None) == -1                            # keys present, pointer missing
+    assert call_ext(lib, B=1 << 16, Hkv=2, Nk=1 << 16) == -2      # key rows overflow int32
+    assert call_ext(lib, q=None, k=None, v=None, o=None, lse=None, Nq=0) == 0   # no queries: empty
+    assert call_ext(lib, q=None, k=None, v=None, o=None, lse=None, B=0) == 0
+

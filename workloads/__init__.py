@@ -16,6 +16,11 @@ Workloads
 ``local_b2_h16_n32k_d128_w4k_cap50``  B=2, H=16, N=32768, d=128, bf16, causal sliding
     window of 4096 keys, logit soft-cap 50, N(0,1) inputs.
 
+Further workloads (``EXTRA_WORKLOADS``) for the general entry point: the local workload
+with 4 attention sinks ("Module 16", section 16.6); a chunk of 1024 new queries against
+a 16384-key cache (the queries are the last 1024 positions, causal); and one decoding
+step (one query row per head) against a 16384-key cache, grouped-query heads.
+
 Random inputs are drawn on the CPU with ``torch.Generator().manual_seed(seed)`` as fp32
 N(0,1), optionally multiplied by a constant in fp32, then rounded to bf16 (round to
 nearest even), so the oracle and the GPU see bit-identical values.  Seeds are
@@ -44,6 +49,12 @@ class Workload:
     softcap: float
     q_mult: float = 1.0
     modular: bool = False
+    nq: int = 0       # query rows per head when they differ from the N key rows (0: N)
+    n_sink: int = 0   # attention sinks beside the window
+
+    @property
+    def Nq(self) -> int:
+        return self.nq if self.nq > 0 else self.N
 
     @property
     def scale(self) -> float:
@@ -58,9 +69,14 @@ class Workload:
         return base, base + 1, base + 2
 
     def describe(self) -> dict:
-        return {"workload": self.name, "B": self.B, "Hq": self.Hq, "Hkv": self.Hkv, "N": self.N,
-                "d": self.d, "dtype": self.dtype, "causal": self.causal, "window": self.window,
-                "softcap": self.softcap, "q_mult": self.q_mult}
+        d = {"workload": self.name, "B": self.B, "Hq": self.Hq, "Hkv": self.Hkv, "N": self.N,
+             "d": self.d, "dtype": self.dtype, "causal": self.causal, "window": self.window,
+             "softcap": self.softcap, "q_mult": self.q_mult}
+        if self.nq > 0:
+            d["Nq"] = self.nq
+        if self.n_sink > 0:
+            d["n_sink"] = self.n_sink
+        return d
 
 
 WORKLOADS = {
@@ -73,6 +89,16 @@ WORKLOADS = {
         Workload("local_b2_h16_n32k_d128_w4k_cap50", 5, 2, 16, 16, 32768, 128, "bfloat16", True, 4096, 50.0),
     ]
 }
+EXTRA_WORKLOADS = {
+    w.name: w
+    for w in [
+        Workload("sink4_b2_h16_n32k_d128_w4k_cap50", 6, 2, 16, 16, 32768, 128, "bfloat16", True, 4096, 50.0,
+                 n_sink=4),
+        Workload("chunk_b4_h32kv8_q1k_k16k_d128", 7, 4, 32, 8, 16384, 128, "bfloat16", True, 0, 0.0, nq=1024),
+        Workload("decode_b32_h32kv8_q1_k16k_d128", 8, 32, 32, 8, 16384, 128, "bfloat16", True, 0, 0.0, nq=1),
+    ]
+}
+ALL_WORKLOADS = {**WORKLOADS, **EXTRA_WORKLOADS}
 BY_NUMBER = {w.number: w for w in WORKLOADS.values()}
 HEADLINE = "causal_b8_h32_n4k_d128"
 
@@ -95,7 +121,7 @@ def _randn(shape, seed: int, mult: float, dtype: torch.dtype) -> torch.Tensor:
 
 
 def make_inputs(w: Workload, seeds=None):
-    """(q, k, v) CPU tensors for workload ``w``: q [B,Hq,N,d], k/v [B,Hkv,N,d]."""
+    """(q, k, v) CPU tensors for workload ``w``: q [B,Hq,Nq,d], k/v [B,Hkv,N,d]."""
     if w.modular:
         if (w.B, w.Hq, w.Hkv) != (1, 1, 1):
             raise ValueError("modular inputs are defined for one head")
@@ -106,7 +132,7 @@ def make_inputs(w: Workload, seeds=None):
         return q.to(dt), k.to(dt), v.to(dt)
     dt = torch.bfloat16 if w.dtype == "bfloat16" else torch.float32
     sq, sk, sv = seeds if seeds is not None else w.seeds()
-    q = _randn((w.B, w.Hq, w.N, w.d), sq, w.q_mult, dt)
+    q = _randn((w.B, w.Hq, w.Nq, w.d), sq, w.q_mult, dt)
     k = _randn((w.B, w.Hkv, w.N, w.d), sk, 1.0, dt)
     v = _randn((w.B, w.Hkv, w.N, w.d), sv, 1.0, dt)
     return q, k, v
@@ -118,12 +144,20 @@ def random_inputs(B, Hq, Hkv, N, d, dtype="bfloat16", seed=0, q_mult=1.0):
     return make_inputs(w, seeds=(seed, seed + 1, seed + 2))
 
 
+def random_cross_inputs(B, Hq, Hkv, Nq, Nk, d, dtype="bfloat16", seed=0, q_mult=1.0):
+    """(q, k, v) with Nq query rows and Nk key rows per head (tests): q [B,Hq,Nq,d] from
+    ``seed``, k and v [B,Hkv,Nk,d] from ``seed + 1`` and ``seed + 2``."""
+    dt = torch.bfloat16 if dtype == "bfloat16" else torch.float32
+    return (_randn((B, Hq, Nq, d), seed, q_mult, dt), _randn((B, Hkv, Nk, d), seed + 1, 1.0, dt),
+            _randn((B, Hkv, Nk, d), seed + 2, 1.0, dt))
+
+
 def sample_rows(w: Workload, per_head_rows, heads=None):
-    """Flat row indices (b*Hq + hq)*N + i for the given query rows of the given heads
+    """Flat row indices (b*Hq + hq)*Nq + i for the given query rows of the given heads
     (all heads by default)."""
     heads = range(w.B * w.Hq) if heads is None else heads
-    rows = sorted(set(int(i) for i in per_head_rows if 0 <= int(i) < w.N))
-    return np.array([bh * w.N + i for bh in heads for i in rows], dtype=np.int64)
+    rows = sorted(set(int(i) for i in per_head_rows if 0 <= int(i) < w.Nq))
+    return np.array([bh * w.Nq + i for bh in heads for i in rows], dtype=np.int64)
 
 
 def standard_row_sample(N: int, head: int = 256, tail: int = 256, stride: int = 61):
@@ -132,5 +166,5 @@ def standard_row_sample(N: int, head: int = 256, tail: int = 256, stride: int = 
     return sorted(s)
 
 
-__all__ = ["Workload", "WORKLOADS", "BY_NUMBER", "HEADLINE", "make_inputs", "random_inputs",
+__all__ = ["Workload", "WORKLOADS", "EXTRA_WORKLOADS", "ALL_WORKLOADS", "BY_NUMBER", "HEADLINE", "make_inputs", "random_inputs", "random_cross_inputs",
            "modular_matrix", "sample_rows", "standard_row_sample"]
