@@ -43,6 +43,31 @@ int current_device(int* dev) {
   return FA_OK;
 }
 
+template <int D, bool kSplit, bool kSinks>
+cudaError_t set_tc_smem() {
+  return cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              fa::tc::Layout<D>::kSmemLaunch);
+}
+
+template <int D, bool kSplit, bool kSinks>
+void launch_tc_kernel(unsigned grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const fa::tc::Params& p, cudaStream_t s) {
+  fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks><<<grid, fa::tc::kThreads, fa::tc::Layout<D>::kSmemLaunch, s>>>(mq, mk, mv,
+                                                                                                            p);
+}
+
+template <int D>
+void launch_tc_variant(bool split, bool sinks, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mk,
+                       const CUtensorMap& mv, const fa::tc::Params& p, cudaStream_t s) {
+  if (split) {
+    if (sinks) launch_tc_kernel<D, true, true>(grid, mq, mk, mv, p, s);
+    else launch_tc_kernel<D, true, false>(grid, mq, mk, mv, p, s);
+  } else {
+    if (sinks) launch_tc_kernel<D, false, true>(grid, mq, mk, mv, p, s);
+    else launch_tc_kernel<D, false, false>(grid, mq, mk, mv, p, s);
+  }
+}
+
 int prepare_device(int dev, int* num_sms = nullptr) {
   DeviceState& st = g_dev[dev];
   std::call_once(st.once, [&] {
@@ -58,17 +83,14 @@ int prepare_device(int dev, int* num_sms = nullptr) {
     }
     st.num_sms = prop.multiProcessorCount;
 
-    e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fa::tc::Layout<128>::kSmemLaunch);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::tc::Layout<64>::kSmemLaunch);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::tc::Layout<128>::kSmemLaunch);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::tc::Layout<64>::kSmemLaunch);
+    e = set_tc_smem<128, false, false>();
+    if (e == cudaSuccess) e = set_tc_smem<128, true, false>();
+    if (e == cudaSuccess) e = set_tc_smem<128, false, true>();
+    if (e == cudaSuccess) e = set_tc_smem<128, true, true>();
+    if (e == cudaSuccess) e = set_tc_smem<64, false, false>();
+    if (e == cudaSuccess) e = set_tc_smem<64, true, false>();
+    if (e == cudaSuccess) e = set_tc_smem<64, false, true>();
+    if (e == cudaSuccess) e = set_tc_smem<64, true, true>();
     // the fp32 path needs up to 4 * (32 d + 32 (d + 1) + 32 d) bytes = 49280 at d = 128
     const int f32_smem = 64 * 1024;
     if (e == cudaSuccess)
@@ -231,17 +253,11 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.n_units = static_cast<int>(units);
   // persistent: one CTA per SM (never more CTAs than units)
   const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
-  if (d == 128) {
-    if (split)
-      tc::fa_fwd_tc_kernel<128, true><<<grid, tc::kThreads, tc::Layout<128>::kSmemLaunch, s>>>(mq, mk, mv, p);
-    else
-      tc::fa_fwd_tc_kernel<128, false><<<grid, tc::kThreads, tc::Layout<128>::kSmemLaunch, s>>>(mq, mk, mv, p);
-  } else {
-    if (split)
-      tc::fa_fwd_tc_kernel<64, true><<<grid, tc::kThreads, tc::Layout<64>::kSmemLaunch, s>>>(mq, mk, mv, p);
-    else
-      tc::fa_fwd_tc_kernel<64, false><<<grid, tc::kThreads, tc::Layout<64>::kSmemLaunch, s>>>(mq, mk, mv, p);
-  }
+  const bool sinks = p.n_sink > 0;
+  if (d == 128)
+    launch_tc_variant<128>(split, sinks, grid, mq, mk, mv, p, s);
+  else
+    launch_tc_variant<64>(split, sinks, grid, mq, mk, mv, p, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   if (split) {

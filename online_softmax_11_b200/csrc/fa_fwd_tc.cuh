@@ -243,19 +243,27 @@ __device__ __forceinline__ float make_p(const float (&s)[kHalf], uint32_t taddr_
 }
 
 // 64 scores of the row (tile columns c0 .. c0+63) from TMEM, masked when the tile needs a
-// mask: -inf above column c_hi and in the hole [h_lo, h_hi) (the columns below the window
-// that are not attention sinks; h_lo = 0 without sinks).
-__device__ __forceinline__ void load_half(uint32_t taddr, int c0, bool need_mask, int h_lo, int h_hi, int c_hi,
-                                          float (&s)[kHalf]) {
+// mask: -inf above column c_hi and in the hole [h_lo, h_hi) of columns below the window
+// that are not attention sinks.  sink_cols (uniform over the tile) says whether the tile
+// holds sink columns at all; without them the hole starts at column 0.  kSinks = false
+// (no sinks in the launch) compiles only that second form.
+template <bool kSinks>
+__device__ __forceinline__ void load_half(uint32_t taddr, int c0, bool need_mask, bool sink_cols, int h_lo,
+                                          int h_hi, int c_hi, float (&s)[kHalf]) {
   uint32_t r[kHalf];
   tmem_ld64_wait(taddr, r);
 #pragma unroll
   for (int c = 0; c < kHalf; ++c) s[c] = __uint_as_float(r[c]);
   if (need_mask) {
-    const uint32_t hole = static_cast<uint32_t>(h_hi - h_lo);
+    if (kSinks && sink_cols) {
+      const uint32_t hole = static_cast<uint32_t>(h_hi - h_lo);
 #pragma unroll
-    for (int c = 0; c < kHalf; ++c)
-      s[c] = (static_cast<uint32_t>(c0 + c - h_lo) < hole || c0 + c > c_hi) ? -CUDART_INF_F : s[c];
+      for (int c = 0; c < kHalf; ++c)
+        s[c] = (static_cast<uint32_t>(c0 + c - h_lo) < hole || c0 + c > c_hi) ? -CUDART_INF_F : s[c];
+    } else {
+#pragma unroll
+      for (int c = 0; c < kHalf; ++c) s[c] = (c0 + c < h_hi || c0 + c > c_hi) ? -CUDART_INF_F : s[c];
+    }
   }
 }
 
@@ -266,9 +274,6 @@ struct TileSet {
   int a0, a1, b0, b1;
   __device__ int count() const { return (a1 - a0) + (b1 - b0); }
   __device__ int at(int n) const { return n < a1 - a0 ? a0 + n : b0 + (n - (a1 - a0)); }
-  __device__ bool has(int j) const { return (j >= a0 && j < a1) || (j >= b0 && j < b1); }
-  __device__ int first() const { return a1 > a0 ? a0 : b0; }
-  __device__ int last() const { return b1 > b0 ? b1 - 1 : a1 - 1; }
 };
 
 __device__ __forceinline__ void run_and(int x0, int x1, int y0, int y1, int& r0, int& r1) {
@@ -405,7 +410,11 @@ __device__ __forceinline__ void for_each_tile(const Params& p, F&& f) {
   }
 }
 
-template <int D, bool kSplit>
+// kSplit: write fp32 partials for the split-KV merge instead of O and LSE.
+// kSinks: the launch has attention sinks (a separate run of sink tiles may precede the
+// window's tiles); without them every key-tile set is one run and the loops are the
+// plain ranges.
+template <int D, bool kSplit, bool kSinks>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -522,10 +531,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TileRange& t = w.tr(i);
         uint32_t o_acc = 0;
         const int T = w.ks.count();
-        const int t_first = t.ks.first(), t_last = t.ks.last();
+        // this query tile's key tiles as positions in the work tile's sequence: each of
+        // its runs lies inside one run of the sequence, so it is a run of positions too
+        int sa0 = 0, sa1 = 0, sb0 = 0, sb1 = 0;
+        if constexpr (kSinks) {
+          const int na = w.ks.a1 - w.ks.a0;
+          if (t.ks.a1 > t.ks.a0) {
+            sa0 = (t.ks.a0 >= w.ks.a0 && t.ks.a0 < w.ks.a1) ? t.ks.a0 - w.ks.a0 : na + (t.ks.a0 - w.ks.b0);
+            sa1 = sa0 + (t.ks.a1 - t.ks.a0);
+          }
+          if (t.ks.b1 > t.ks.b0) {
+            sb0 = (t.ks.b0 >= w.ks.a0 && t.ks.b0 < w.ks.a1) ? t.ks.b0 - w.ks.a0 : na + (t.ks.b0 - w.ks.b0);
+            sb1 = sb0 + (t.ks.b1 - t.ks.b0);
+          }
+        } else if (t.ks.b1 > t.ks.b0) {  // one run each
+          sb0 = t.ks.b0 - w.ks.b0;
+          sb1 = t.ks.b1 - w.ks.b0;
+        }
+        const int n_first = sa1 > sa0 ? sa0 : sb0;
+        const int n_last = sb1 > sb0 ? sb1 - 1 : sa1 - 1;
         for (int n = 0; n <= T; ++n) {
-          const int j = n < T ? w.ks.at(n) : -1;       // key tile whose S is issued now
-          const int jp = n > 0 ? w.ks.at(n - 1) : -1;  // key tile whose P.V is issued now
+          // position n: S of the n-th key tile; position n - 1: its P.V
+          const bool use_s = n < T && ((kSinks && n >= sa0 && n < sa1) || (n >= sb0 && n < sb1));
+          const bool use_pv = n > 0 && ((kSinks && n - 1 >= sa0 && n - 1 < sa1) || (n - 1 >= sb0 && n - 1 < sb1));
           const int kidx = used + 2 * n;
           const int vidx = kidx - 1;
           const int kslot = kidx % L::kStages;
@@ -534,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // proxy on shared memory).  P, written to tensor memory by the softmax warps'
           // tcgen05.st, also needs tcgen05.fence::after_thread_sync after its barrier.
           if (n > 0) {
-            if (t.part && t.ks.has(jp)) {
+            if (use_pv) {
               if (!mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
               if (!mbar_wait(&bars[L::kBarPFull + i], p_phase, ctl)) return false;
               p_phase ^= 1u;
@@ -543,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               // of V (128 B each); the two 64-column slabs of V are kHalfBytes apart
               mma_ts_kloop8(d_o, d_s, dvring + ((vslot * L::kTileBytes) >> 4), kIdescPV, o_acc);
               o_acc = 1;
-              if (jp == t_last) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
+              if (n - 1 == n_last) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
               mma_commit(&bars[L::kBarKvEmpty + vslot]);
             } else {
               // not used by this query tile: release it, but only once this fill has
@@ -553,15 +581,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (n < T) {
-            if (t.part && t.ks.has(j)) {
+            if (use_s) {
               if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
-              if (j == t_first) {  // first use of this work tile's Q_i
+              if (n == n_first) {  // first use of this work tile's Q_i
                 if (!mbar_wait(&bars[L::kBarQFull + i], q_cnt & 1u, ctl)) return false;
                 ++q_cnt;
               }
               mma_ss_kloop<D / 16>(d_s, dq, dring + ((kslot * L::kTileBytes) >> 4), kIdescS);
               mma_commit(&bars[L::kBarSFull + i]);
-              if (j == t_last) mma_commit(&bars[L::kBarQEmpty + i]);  // Q_i no longer read
+              if (n == n_last) mma_commit(&bars[L::kBarQEmpty + i]);  // Q_i no longer read
               mma_commit(&bars[L::kBarKvEmpty + kslot]);
             } else {
               if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
@@ -598,9 +626,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float lr = 0.f;           // normaliser of O (l with each tile maximum's P as rounded)
       bool o_valid = false;
 
-      const int T = t.ks.count();
-      for (int n = 0; n < T; ++n) {
-        const int j = t.ks.at(n);
+      // the query tile's key tiles: the sink run, then the window run
+      for (int run = kSinks ? 0 : 1; run < 2; ++run)
+      for (int j = run == 0 ? t.ks.a0 : t.ks.b0, j_end = run == 0 ? t.ks.a1 : t.ks.b1; j < j_end; ++j) {
         // tcgen05.ld/st are warp-collective: the whole warp leaves together or not at all
         if (!__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarSFull + i], s_phase, ctl))) return false;
         s_phase ^= 1u;
@@ -615,6 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int c_hi = min(BN - 1, p.Nk - 1 - k0);
         if (p.causal) c_hi = min(c_hi, pos - k0);
         const int w_lo = p.window > 0 ? max(0, pos - p.window + 1 - k0) : 0;  // window's first column
+        const bool sink_cols = kSinks && p.n_sink > k0;
         const int h_lo = min(max(0, p.n_sink - k0), w_lo);
         const int h_hi = w_lo;
 
@@ -628,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float s[kHalf];
-          load_half(lane_base + colS + h * kHalf, h * kHalf, need_mask, h_lo, h_hi, c_hi, s);
+          load_half<kSinks>(lane_base + colS + h * kHalf, h * kHalf, need_mask, sink_cols, h_lo, h_hi, c_hi, s);
 #pragma unroll
           for (int c = 0; c < kHalf; c += 8) {
             mx0 = fmax3(mx0, s[c], s[c + 1]);
@@ -690,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float s[kHalf];
-          load_half(lane_base + colS + h * kHalf, h * kHalf, need_mask, h_lo, h_hi, c_hi, s);
+          load_half<kSinks>(lane_base + colS + h * kHalf, h * kHalf, need_mask, sink_cols, h_lo, h_hi, c_hi, s);
           const uint32_t tp = lane_base + colS + h * (kHalf / 2);
           if (!p.use_softcap) {
             if (need_mask)
