@@ -25,6 +25,10 @@ Contents
     (query, key) pair; the closed forms 4 B Hq N^2 d, halved for causal, and
     4 B Hq d (N W - W^2/2) for a causal window are reported beside it).
 
+``softmax.softmax(x)``, ``softmax.softmax_topk(x, k)``
+    The classical softmax of each row in fp64 and its top-K with probabilities
+    ("Online normalizer calculation for softmax"; see ``oracle/softmax.py``).
+
 Every function is pinned by ``tests/test_oracle_pins.py`` against values the pages
 print, closed forms, invariants and a library softmax.
 """
