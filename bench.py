@@ -22,6 +22,11 @@ number of kernel launches in the timed region.
 
 ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only), as the reference
 arm of the comparison.
+
+``--op softmax`` / ``--op softmax_topk`` time the stand-alone softmax (online normaliser)
+and the fused softmax + top-K instead, on a softmax workload (default 4096 rows of 32000
+fp32 logits); their metric is HBM bandwidth: bytes that must cross HBM (the row read once
+and, for softmax, written once; K probabilities and indices for top-K) per second.
 """
 from __future__ import annotations
 
@@ -429,13 +434,174 @@ def gpu_arm(args, w):
     return 0
 
 
+SOFTMAX_METRIC = {"softmax": "stand-alone softmax GB/s (rows read and written once) on 1 B200",
+                  "softmax_topk": "fused softmax + top-K GB/s (rows read once) on 1 B200"}
+
+
+def softmax_bytes(sw, op: str) -> float:
+    """Bytes that must cross HBM per step: x read once; y written (softmax) or K
+    probabilities + K int32 indices (top-K); one fp32 LSE per row."""
+    out = sw.rows * sw.V * 4 if op == "softmax" else sw.rows * sw.k * 8
+    return float(sw.rows * sw.V * 4 + out + sw.rows * 4)
+
+
+def softmax_oracle_time(sw, op: str, x, seconds: float, offset: int = 0):
+    """The fp64 oracle on a bounded row sample: returns (GB/s of the same accounting,
+    seconds, rows, threads=1: numpy on one core)."""
+    from oracle import softmax as osm
+    t0 = time.perf_counter()
+    osm.softmax(x[:4]) if op == "softmax" else osm.softmax_topk(x[:4], sw.k)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    n = int(max(1, min(sw.rows, 4 * seconds / dt)))
+    start = (offset * 97) % max(1, sw.rows - n + 1)
+    t0 = time.perf_counter()
+    osm.softmax(x[start:start + n]) if op == "softmax" else osm.softmax_topk(x[start:start + n], sw.k)
+    dt = time.perf_counter() - t0
+    return softmax_bytes(sw, op) * n / sw.rows / dt / 1e9, dt, n
+
+
+def softmax_arm(args, sw):
+    """Time fa_softmax / fa_softmax_topk (ours) or the oracle (reference) on ``sw``."""
+    import torch
+    op = args.op
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        x = workloads.make_logits(sw)
+        total_b, total_s = 0.0, 0.0
+        budget = float(args.reference_seconds) / max(1, args.steps + args.warmup)
+        for step in range(args.warmup + args.steps):
+            gbs, dt, n = softmax_oracle_time(sw, op, x, budget, step)
+            if step >= args.warmup:
+                total_b += gbs * dt
+                total_s += dt
+        value = total_b / total_s
+        sample = f"{n} of {sw.rows} rows per step, numpy fp64 on one core"
+        emit({"impl": "reference", "metric": SOFTMAX_METRIC[op], "value": value, "unit": "GB/s", "n_gpus": ws,
+              "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_s / args.steps * 1e3,
+              "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+              "config": sw.describe(),
+              "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+              "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+        return 0
+    import torch.distributed as dist
+    import online_softmax_11_b200 as fa
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+    lib = fa.load()
+    x_h = workloads.make_logits(sw, seed=sw.seed + 100 * rank)
+    x = x_h.to(dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    y = torch.empty_like(x)
+    probs = torch.empty((sw.rows, sw.k), dtype=torch.float32, device=dev)
+    idx = torch.empty((sw.rows, sw.k), dtype=torch.int32, device=dev)
+    lse = torch.empty(sw.rows, dtype=torch.float32, device=dev)
+
+    def step(xx):
+        if op == "softmax":
+            rc = lib.fa_softmax(xx.data_ptr(), y.data_ptr(), lse.data_ptr(), sw.rows, sw.V, sh)
+        else:
+            rc = lib.fa_softmax_topk(xx.data_ptr(), probs.data_ptr(), idx.data_ptr(), lse.data_ptr(), sw.rows, sw.V,
+                                     sw.k, sh)
+        if rc != 0:
+            raise fa.FAError(rc, lib, "fa_" + op)
+
+    for _ in range(args.warmup):
+        step(x)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local if ws > 1 else 0) if not args.no_clocks else None
+    if sampler is not None:
+        time.sleep(0.3)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(x)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    if ws > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    clocks = sampler.stop() if sampler is not None else None
+    max_ms = max_over_ranks(ms, dev)
+    nbytes = softmax_bytes(sw, op)
+    value = ws * nbytes * args.steps / (max_ms / 1e3) / 1e9
+    per_launch = ms / args.steps
+
+    e2e = None
+    if not args.no_e2e:
+        xp = x_h.pin_memory()
+        outp = torch.empty(y.shape if op == "softmax" else probs.shape, dtype=torch.float32, pin_memory=True)
+        ip = torch.empty(idx.shape, dtype=torch.int32, pin_memory=True)
+        xd = torch.empty_like(x)
+
+        def e2e_step():
+            xd.copy_(xp, non_blocking=True)
+            step(xd)
+            if op == "softmax":
+                outp.copy_(y, non_blocking=True)
+            else:
+                outp.copy_(probs, non_blocking=True)
+                ip.copy_(idx, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(1, min(args.e2e_steps, args.steps))
+        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        es.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        ee.record(stream)
+        torch.cuda.synchronize(dev)
+        te = max_over_ranks(es.elapsed_time(ee), dev)
+        d2h = y.numel() * 4 if op == "softmax" else probs.numel() * 4 + idx.numel() * 4
+        e2e = {"value": ws * nbytes * n_e2e / (te / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": x.numel() * 4,
+               "d2h_bytes_per_step": d2h, "steps": n_e2e, "ms_per_step": te / n_e2e}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        gbs, secs, n = softmax_oracle_time(sw, op, x_h, min(args.cpu_seconds, 10.0))
+        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{n} of {sw.rows} rows, numpy fp64 on one core, {secs:.1f} s"}
+    peaks, src = load_peaks()
+    peak_bw = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    achieved = nbytes / (per_launch / 1e3) / 1e9
+    kmax = next(c for c in (4, 8, 16, 32) if sw.k <= c)
+    kernel = "softmax_online_kernel" if op == "softmax" else f"softmax_topk_kernel<{kmax}>"
+    if rank == 0:
+        emit({"metric": SOFTMAX_METRIC[op], "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+              "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+              "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+              "config": {**sw.describe(), "l2": "inputs larger than L2 (no flush needed)",
+                         "parallelism": f"replicas x{ws} (independent batches)"},
+              "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
+                           "frac": achieved / peak_bw, "traffic": None, "peak_source": f"hbm_gbs of {src}",
+                           "kernel": kernel, "algorithmic_bytes_per_launch": nbytes},
+              "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": args.steps})
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.ALL_WORKLOADS))
+    ap.add_argument("--op", choices=["attention", "softmax", "softmax_topk"], default="attention")
+    ap.add_argument("--workload", default=None,
+                    choices=sorted(workloads.ALL_WORKLOADS) + sorted(workloads.SOFTMAX_WORKLOADS))
     ap.add_argument("--batch", type=int, default=None, help="override B (profiling on a smaller case)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -447,15 +613,22 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     args = ap.parse_args(argv)
-    w = workloads.ALL_WORKLOADS[args.workload]
-    if w.dtype != "bfloat16" and args.impl == "ours":
-        ap.error("the benchmark times the bf16 tensor-core path")
-    if args.batch is not None:
-        w = w.with_(B=args.batch)
     ws, _, _ = dist_env()
     if args.gpus != ws:
         ap.error(f"--gpus {args.gpus} needs one process per GPU: launch with torchrun --nproc-per-node "
                  f"{args.gpus} (WORLD_SIZE is {ws})")
+    if args.op != "attention":
+        name = args.workload or "softmax_r4k_v32k"
+        if name not in workloads.SOFTMAX_WORKLOADS:
+            ap.error(f"--op {args.op} takes a softmax workload: {sorted(workloads.SOFTMAX_WORKLOADS)}")
+        return softmax_arm(args, workloads.SOFTMAX_WORKLOADS[name])
+    if args.workload in workloads.SOFTMAX_WORKLOADS:
+        ap.error("softmax workloads need --op softmax or --op softmax_topk")
+    w = workloads.ALL_WORKLOADS[args.workload or workloads.HEADLINE]
+    if w.dtype != "bfloat16" and args.impl == "ours":
+        ap.error("the benchmark times the bf16 tensor-core path")
+    if args.batch is not None:
+        w = w.with_(B=args.batch)
     if args.impl == "reference":
         return reference_arm(args, w)
     return gpu_arm(args, w)

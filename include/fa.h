@@ -181,6 +181,37 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
                int Hkv, int N, int d, float scale, int causal, int window, float softcap, void* stream);
 
 /*
+ * fa_softmax -- stand-alone softmax of every row with the online normaliser.
+ * Source: "Online normalizer calculation for softmax" (Milakov and Gimelshein): the
+ * classical softmax, computed with fewer memory accesses by keeping the running maximum
+ * and the normaliser together in one pass (the normaliser is rescaled by
+ * exp(m_old - m_new) when the maximum grows); a second pass writes the outputs.
+ *   x, y : float device arrays [rows, V], row-major, 16-byte aligned, not overlapping.
+ *          y[r, i] = exp(x[r, i] - m_r) / d_r, m_r = max_i x[r, i],
+ *          d_r = sum_i exp(x[r, i] - m_r).
+ *   lse  : float [rows] or NULL: m_r + ln d_r (-inf for V == 0).
+ *   rows, V >= 0.  A row whose inputs are all -inf is undefined (0 / 0).
+ * Precision: fp32 in and out; exponentials as exp2 of x log2(e) (approximate exp2,
+ * relative error about 2^-22), normaliser summed in fp32.
+ * Errors: FA_ERR_BAD_SHAPE (rows or V < 0), FA_ERR_NULL_PTR, FA_ERR_ALIGN, FA_ERR_CUDA.
+ */
+int fa_softmax(const float* x, float* y, float* lse, int rows, int V, void* stream);
+
+/*
+ * fa_softmax_topk -- softmax fused with top-K: one read of each row gives the row's
+ * maximum and normaliser and its K largest inputs (the fused Softmax+TopK of "Online
+ * normalizer calculation for softmax").  Nothing of size V is written.
+ *   x     : float [rows, V], 16-byte aligned.
+ *   probs : float [rows, K]: softmax probabilities exp(x_k - m) / d of the K largest
+ *           inputs, largest first.
+ *   idx   : int [rows, K]: their column indices.  Equal inputs are ordered by lower
+ *           index first (the page does not say; this is the library's rule).
+ *   lse   : float [rows] or NULL, as fa_softmax.
+ *   1 <= K <= 32 and K <= V (FA_ERR_BAD_ARG otherwise).  Other errors as fa_softmax.
+ */
+int fa_softmax_topk(const float* x, float* probs, int* idx, float* lse, int rows, int V, int K, void* stream);
+
+/*
  * fa_check_status -- synchronise `stream`, then report (and clear) the device status
  * word that kernels of this library set when one of their bounded waits ran out
  * (FA_ERR_TIMEOUT) on the current device, or a pending CUDA error (FA_ERR_CUDA).

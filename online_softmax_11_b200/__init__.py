@@ -36,7 +36,7 @@ ERRORS = {
 STATIC_SCRATCH_BYTES = 32 << 20
 MAX_SPLITS = 64
 # every symbol include/fa.h declares
-EXPORTS = ["fa_fwd", "fa_fwd_f32", "fa_fwd_ext", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace", "fa_fwd_splitkv_static",
+EXPORTS = ["fa_fwd", "fa_fwd_f32", "fa_fwd_ext", "fa_softmax", "fa_softmax_topk", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace", "fa_fwd_splitkv_static",
            "fa_check_status", "fa_selftest_wait_timeout", "fa_strerror", "fa_last_cuda_error", "fa_version"]
 
 _lock = threading.Lock()
@@ -78,6 +78,10 @@ def load():
         lib.fa_fwd_splitkv_static.argtypes = sig[:-1] + [i, vp]
         lib.fa_fwd_ext.restype = i
         lib.fa_fwd_ext.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, f, i, vp, ctypes.c_size_t, vp]
+        lib.fa_softmax.restype = i
+        lib.fa_softmax.argtypes = [vp, vp, vp, i, i, vp]
+        lib.fa_softmax_topk.restype = i
+        lib.fa_softmax_topk.argtypes = [vp, vp, vp, vp, i, i, i, vp]
         lib.fa_fwd_splitkv_workspace.restype = ctypes.c_size_t
         lib.fa_fwd_splitkv_workspace.argtypes = [i, i, i, i, i]
         lib.fa_check_status.restype = i
@@ -224,6 +228,46 @@ def forward_ext(q, k, v, *, scale: float | None = None, causal: bool = False, wi
     return out, lse
 
 
+def _check_rows(x, what):
+    import torch
+    if x.dim() != 2 or x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError(f"{what}: x must be a contiguous float32 CUDA tensor [rows, V]")
+
+
+def softmax(x, *, out=None, lse=None, return_lse: bool = False, stream=None):
+    """Row softmax of float32 ``x`` [rows, V] through ``fa_softmax`` (online normaliser)."""
+    import torch
+    _check_rows(x, "fa_softmax")
+    rows, V = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    if return_lse and lse is None:
+        lse = torch.empty(rows, dtype=torch.float32, device=x.device)
+    with torch.cuda.device(x.device):
+        rc = load().fa_softmax(x.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None, rows, V,
+                               _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, load(), "fa_softmax")
+    return (out, lse) if return_lse else out
+
+
+def softmax_topk(x, k: int, *, stream=None):
+    """Fused softmax + top-``k`` of float32 ``x`` [rows, V] through ``fa_softmax_topk``.
+    Returns (probs [rows, k] float32, idx [rows, k] int32, lse [rows] float32)."""
+    import torch
+    _check_rows(x, "fa_softmax_topk")
+    rows, V = x.shape
+    probs = torch.empty((rows, k), dtype=torch.float32, device=x.device)
+    idx = torch.empty((rows, k), dtype=torch.int32, device=x.device)
+    lse = torch.empty(rows, dtype=torch.float32, device=x.device)
+    with torch.cuda.device(x.device):
+        rc = load().fa_softmax_topk(x.data_ptr(), probs.data_ptr(), idx.data_ptr(), lse.data_ptr(), rows, V, int(k),
+                                    _stream_handle(stream))
+    if rc != FA_OK:
+        raise FAError(rc, load(), "fa_softmax_topk")
+    return probs, idx, lse
+
+
 def check_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return load().fa_check_status(_stream_handle(stream))
@@ -245,5 +289,5 @@ def attention_flops(B: int, Hq: int, N: int, d: int, causal: bool = False, windo
     return 4.0 * d * B * Hq * pairs
 
 
-__all__ = ["forward", "forward_ext", "forward_splitkv", "splitkv_workspace_bytes", "fwd_raw", "load", "check_status",
+__all__ = ["forward", "forward_ext", "forward_splitkv", "softmax", "softmax_topk", "splitkv_workspace_bytes", "fwd_raw", "load", "check_status",
            "selftest_wait_timeout", "attention_flops", "FAError", "EXPORTS", "LIB_PATH", "MAX_SPLITS"]

@@ -12,6 +12,7 @@
 #include "fa_fwd_f32.cuh"
 #include "fa_fwd_tc.cuh"
 #include "fa_merge.cuh"
+#include "fa_softmax.cuh"
 
 namespace {
 
@@ -91,6 +92,8 @@ int prepare_device(int dev, int* num_sms = nullptr) {
     if (e == cudaSuccess) e = set_tc_smem<64, true, false>();
     if (e == cudaSuccess) e = set_tc_smem<64, false, true>();
     if (e == cudaSuccess) e = set_tc_smem<64, true, true>();
+    if (e == cudaSuccess)  // two 1024-thread softmax blocks per SM: keep L1 small, shared memory is tiny
+      e = cudaFuncSetAttribute(fa::smx::softmax_online_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 10);
     // the fp32 path needs up to 4 * (32 d + 32 (d + 1) + 32 d) bytes = 49280 at d = 128
     const int f32_smem = 64 * 1024;
     if (e == cudaSuccess)
@@ -482,6 +485,53 @@ int fa_selftest_wait_timeout(unsigned timeout_us, void* stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return fa_check_status(stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// stand-alone softmax (online normaliser) and softmax + top-K
+// ---------------------------------------------------------------------------------
+extern "C" {
+
+int fa_softmax(const float* x, float* y, float* lse, int rows, int V, void* stream) {
+  if (rows < 0 || V < 0) return FA_ERR_BAD_SHAPE;
+  if (rows == 0) return FA_OK;
+  if (V > 0 && (!x || !y)) return FA_ERR_NULL_PTR;  // V == 0: nothing is read, only lse is written
+  if (!aligned(x, 16) || !aligned(y, 16) || (lse && !aligned(lse, 4))) return FA_ERR_ALIGN;
+  int dev, rc;
+  if ((rc = current_device(&dev)) != FA_OK) return rc;
+  if ((rc = prepare_device(dev)) != FA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // 1024 threads for long rows; short rows do not need that many
+  const int threads = V >= 16384 ? fa::smx::kSoftmaxThreads : 256;
+  fa::smx::softmax_online_kernel<<<static_cast<unsigned>(rows), threads, 0, s>>>(x, y, lse, V);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int fa_softmax_topk(const float* x, float* probs, int* idx, float* lse, int rows, int V, int K, void* stream) {
+  if (rows < 0 || V < 0) return FA_ERR_BAD_SHAPE;
+  if (K < 1 || K > fa::smx::kMaxTopK || (rows > 0 && K > V)) return FA_ERR_BAD_ARG;
+  if (rows == 0) return FA_OK;
+  if (!x || !probs || !idx) return FA_ERR_NULL_PTR;
+  if (!aligned(x, 16) || !aligned(probs, 4) || !aligned(idx, 4) || (lse && !aligned(lse, 4))) return FA_ERR_ALIGN;
+  int dev, rc;
+  if ((rc = current_device(&dev)) != FA_OK) return rc;
+  if ((rc = prepare_device(dev)) != FA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned g = static_cast<unsigned>(rows);
+  constexpr int T = fa::smx::kTopkThreads;
+  if (K <= 4)
+    fa::smx::softmax_topk_kernel<4><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
+  else if (K <= 8)
+    fa::smx::softmax_topk_kernel<8><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
+  else if (K <= 16)
+    fa::smx::softmax_topk_kernel<16><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
+  else
+    fa::smx::softmax_topk_kernel<32><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
 }  // extern "C"

@@ -160,3 +160,18 @@ def test_ext_argument_errors(lib):
     assert call_ext(lib, q=None, k=None, v=None, o=None, lse=None, Nq=0) == 0   # no queries: empty
     assert call_ext(lib, q=None, k=None, v=None, o=None, lse=None, B=0) == 0
 
+
+def test_softmax_argument_errors(lib):
+    assert lib.fa_softmax(FAKE, FAKE, None, -1, 8, None) == -2
+    assert lib.fa_softmax(FAKE, FAKE, None, 2, -8, None) == -2
+    assert lib.fa_softmax(None, FAKE, None, 2, 8, None) == -1
+    assert lib.fa_softmax(FAKE + 4, FAKE, None, 2, 8, None) == -4
+    assert lib.fa_softmax(FAKE, FAKE + 8, None, 2, 8, None) == -4
+    assert lib.fa_softmax(None, None, None, 0, 8, None) == 0      # no rows
+    assert lib.fa_softmax_topk(FAKE, FAKE, FAKE, None, 2, 8, 0, None) == -5
+    assert lib.fa_softmax_topk(FAKE, FAKE, FAKE, None, 2, 8, 9, None) == -5     # K > V
+    assert lib.fa_softmax_topk(FAKE, FAKE, FAKE, None, 2, 100, 33, None) == -5  # K > 32
+    assert lib.fa_softmax_topk(FAKE, None, FAKE, None, 2, 100, 4, None) == -1
+    assert lib.fa_softmax_topk(FAKE + 4, FAKE, FAKE, None, 2, 100, 4, None) == -4
+    assert lib.fa_softmax_topk(None, None, None, None, 0, 100, 4, None) == 0
+

@@ -16,6 +16,10 @@ Workloads
 ``local_b2_h16_n32k_d128_w4k_cap50``  B=2, H=16, N=32768, d=128, bf16, causal sliding
     window of 4096 keys, logit soft-cap 50, N(0,1) inputs.
 
+Softmax workloads (``SOFTMAX_WORKLOADS``): 4096 rows of 32000 logits and 1024 rows of
+262144 logits, fp32 N(0,1) * 4, top-K with K = 5 (vocabulary-sized rows; the page gives
+no sizes).
+
 Further workloads (``EXTRA_WORKLOADS``) for the general entry point: the local workload
 with 4 attention sinks ("Module 16", section 16.6); a chunk of 1024 new queries against
 a 16384-key cache (the queries are the last 1024 positions, causal); and one decoding
@@ -103,6 +107,35 @@ BY_NUMBER = {w.number: w for w in WORKLOADS.values()}
 HEADLINE = "causal_b8_h32_n4k_d128"
 
 
+@dataclasses.dataclass(frozen=True)
+class SoftmaxWorkload:
+    """Rows of logits for the stand-alone softmax / softmax + top-K: fp32 N(0,1) * scale."""
+    name: str
+    rows: int
+    V: int
+    k: int
+    scale: float = 4.0
+    seed: int = 9000
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "rows": self.rows, "V": self.V, "k": self.k, "dtype": "float32",
+                "values": f"N(0,1) * {self.scale}"}
+
+
+SOFTMAX_WORKLOADS = {
+    w.name: w
+    for w in [
+        SoftmaxWorkload("softmax_r4k_v32k", 4096, 32000, 5),
+        SoftmaxWorkload("softmax_r1k_v256k", 1024, 262144, 5, seed=9100),
+    ]
+}
+
+
+def make_logits(w: SoftmaxWorkload, seed=None) -> torch.Tensor:
+    """[rows, V] fp32 CPU logits for a softmax workload."""
+    return _randn((w.rows, w.V), w.seed if seed is None else seed, w.scale, torch.float32)
+
+
 def modular_matrix(n: int, d: int, a: int, b: int, m: int) -> np.ndarray:
     """nx_flashattn_scale.nx ``fa_seed``: x = (a i + b c) mod m, value (x - m/2) / m with
     integer m/2, converted to fp32 and divided in fp32 (IEEE, correctly rounded)."""
@@ -166,5 +199,5 @@ def standard_row_sample(N: int, head: int = 256, tail: int = 256, stride: int = 
     return sorted(s)
 
 
-__all__ = ["Workload", "WORKLOADS", "EXTRA_WORKLOADS", "ALL_WORKLOADS", "BY_NUMBER", "HEADLINE", "make_inputs", "random_inputs", "random_cross_inputs",
+__all__ = ["SoftmaxWorkload", "SOFTMAX_WORKLOADS", "make_logits", "Workload", "WORKLOADS", "EXTRA_WORKLOADS", "ALL_WORKLOADS", "BY_NUMBER", "HEADLINE", "make_inputs", "random_inputs", "random_cross_inputs",
            "modular_matrix", "sample_rows", "standard_row_sample"]
