@@ -396,8 +396,11 @@ def gpu_arm(args, w):
     peaks, peaks_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_bw = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    kernel = (f"fa_fwd_tc_kernel<{w.d}, {'true' if args.splits > 0 else 'false'}, "
-              f"{'true' if (w.n_sink > 0 and w.window > 0) else 'false'}>")
+    if (w.Hq // w.Hkv) * w.Nq <= 16:  # the group's query rows fit one 16-row block
+        kernel = f"fa_decode_kernel<{w.d}>"
+    else:
+        kernel = (f"fa_fwd_tc_kernel<{w.d}, {'true' if args.splits > 0 else 'false'}, "
+                  f"{'true' if (w.n_sink > 0 and w.window > 0) else 'false'}>")
     # algorithmic bytes: Q, K, V read once, O and LSE written once
     alg_bytes = float(q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size()
                       + o.numel() * o.element_size() + lse.numel() * lse.element_size())

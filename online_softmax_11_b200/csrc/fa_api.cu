@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_decode.cuh"
 #include "fa_fwd_f32.cuh"
 #include "fa_fwd_tc.cuh"
 #include "fa_merge.cuh"
@@ -84,7 +85,12 @@ int prepare_device(int dev, int* num_sms = nullptr) {
     }
     st.num_sms = prop.multiProcessorCount;
 
-    e = set_tc_smem<128, false, false>();
+    e = cudaFuncSetAttribute(fa::dec::fa_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::dec::Smem<128>::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::dec::fa_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::dec::Smem<64>::kAlloc);
+    if (e == cudaSuccess) e = set_tc_smem<128, false, false>();
     if (e == cudaSuccess) e = set_tc_smem<128, true, false>();
     if (e == cudaSuccess) e = set_tc_smem<128, false, true>();
     if (e == cudaSuccess) e = set_tc_smem<128, true, true>();
@@ -130,12 +136,12 @@ EncodeTiledFn encode_fn() {
 // [heads, N, d] bf16 tensor viewed as 3-D (d, N, heads); boxes of 64 columns x 128 rows
 // with 128-byte swizzle, which is the canonical K-major (Q, K) and MN-major (V) operand
 // layout of tcgen05.mma.  Rows past N read as zero.
-int make_map(CUtensorMap* map, const void* base, int heads, int N, int d) {
+int make_map(CUtensorMap* map, const void* base, int heads, int N, int d, unsigned box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(heads)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t elem_strides[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem_strides,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -207,6 +213,66 @@ int launch_no_keys(void* o, float* lse, long long rows, int d, cudaStream_t s) {
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
+// Few query rows per key/value head (the whole group's rows fit one 16-row block): the
+// decode kernel, one block per (batch, key/value head, key chunk).
+int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                  int Nk, int d, float scale, int causal, int window, int n_sink, float softcap, int num_splits,
+                  float* o_part, float* lse_part, cudaStream_t s) {
+  int rc;
+  CUtensorMap mk, mv;
+  if ((rc = make_map(&mk, k, B * Hkv, Nk, d, fa::dec::kKeys)) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * Hkv, Nk, d, fa::dec::kKeys)) != FA_OK) return rc;
+  fa::dec::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.group = Hq / Hkv;
+  p.n_bh = B * Hq;
+  p.causal = causal ? 1 : 0;
+  p.window = window > 0 ? window : 0;
+  p.n_sink = window > 0 ? n_sink : 0;
+  p.scale_log2 = scale * fa::dec::kLog2e;
+  p.use_softcap = softcap > 0.f ? 1 : 0;
+  p.cap_inner = softcap > 0.f ? scale / softcap : 0.f;
+  p.cap_outer = softcap > 0.f ? softcap * fa::dec::kLog2e : 0.f;
+  const bool split = num_splits >= 1;
+  p.num_splits = split ? num_splits : 1;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.timeout_ns = kWaitLimitNs;
+  const long long blocks = static_cast<long long>(B) * Hkv * p.num_splits;
+  if (blocks > 0x7fffffffll) return FA_ERR_BAD_SHAPE;
+  // with one chunk the kernel writes bf16 O / LSE itself; with more, fp32 partials
+  if (p.num_splits == 1) {
+    p.o_part = nullptr;
+    p.lse_part = nullptr;
+  }
+  const unsigned grid = static_cast<unsigned>(blocks);
+  if (d == 128)
+    fa::dec::fa_decode_kernel<128><<<grid, fa::dec::kThreads, fa::dec::Smem<128>::kAlloc, s>>>(mk, mv, p);
+  else
+    fa::dec::fa_decode_kernel<64><<<grid, fa::dec::kThreads, fa::dec::Smem<64>::kAlloc, s>>>(mk, mv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (p.num_splits > 1) {
+    const long long rows = static_cast<long long>(B) * Hq * Nq;
+    const unsigned mgrid = static_cast<unsigned>((rows + fa::kMergeRowsPerBlock - 1) / fa::kMergeRowsPerBlock);
+    if (d == 128)
+      fa::fa_merge_splits_kernel<128><<<mgrid, 32 * fa::kMergeRowsPerBlock, 0, s>>>(
+          o_part, lse_part, static_cast<__nv_bfloat16*>(o), lse, rows, num_splits);
+    else
+      fa::fa_merge_splits_kernel<64><<<mgrid, 32 * fa::kMergeRowsPerBlock, 0, s>>>(
+          o_part, lse_part, static_cast<__nv_bfloat16*>(o), lse, rows, num_splits);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return FA_OK;
+}
+
 // Launch the tensor-core kernel: plain (num_splits == 0: bf16 O and fp32 LSE) or split-KV
 // (num_splits >= 1: fp32 partials into o_part / lse_part, then the merge kernel).
 int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
@@ -217,6 +283,9 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   if ((rc = current_device(&dev)) != FA_OK) return rc;
   if ((rc = prepare_device(dev, &num_sms)) != FA_OK) return rc;
   if (Nk == 0) return launch_no_keys(o, lse, static_cast<long long>(B) * Hq * Nq, d, s);
+  if ((Hq / Hkv) * static_cast<long long>(Nq) <= fa::dec::kRows)
+    return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, n_sink, softcap, num_splits,
+                         o_part, lse_part, s);
 
   CUtensorMap mq, mk, mv;
   if ((rc = make_map(&mq, q, B * Hq, Nq, d)) != FA_OK) return rc;

@@ -79,6 +79,16 @@ CASES = [
     (1, 2, 2, 1100, 1100, 128, True, 128, 4, 0.0, 3),  # sinks with split-KV
     (1, 2, 1, 600, 2500, 128, True, 300, 4, 0.0, 2),   # all of it at once
     (1, 2, 2, 300, 300, 128, False, 0, 4, 0.0, 0),     # sinks without a window: no effect
+    # few query rows per key/value head (group x Nq <= 16): the decode kernel
+    (2, 32, 8, 1, 4099, 128, True, 0, 0, 0.0, 0),     # one decoding step, GQA 4
+    (2, 32, 8, 4, 1000, 128, True, 0, 0, 0.0, 0),     # 16 rows: 4 heads x 4 queries
+    (1, 16, 2, 2, 777, 64, True, 0, 0, 0.0, 3),       # 16 rows, d = 64, split-KV
+    (1, 8, 8, 3, 20, 128, True, 0, 0, 0.0, 0),        # fewer keys than one tile
+    (1, 8, 8, 5, 3, 128, True, 0, 0, 0.0, 0),         # more queries than keys: empty rows
+    (1, 4, 1, 4, 3000, 128, True, 512, 4, 0.0, 2),    # window + sinks
+    (1, 4, 2, 2, 2000, 128, True, 300, 0, 30.0, 0),   # window + soft-cap
+    (1, 4, 4, 1, 1500, 64, False, 0, 0, 0.0, 0),      # non-causal cross-attention
+    (1, 2, 1, 7, 40000, 128, True, 0, 0, 0.0, 5),     # long cache, split-KV
 ]
 
 
@@ -133,3 +143,22 @@ def test_ext_sinks_full_size_local_workload(fa):
                                 rows=rows)
     rt = torch.from_numpy(rows).to(dev)
     compare_rows(o.reshape(-1, w.d)[rt].double().cpu().numpy(), lse.reshape(-1)[rt].double().cpu().numpy(), ro, rlse)
+
+
+def test_decode_full_size_workload(fa):
+    """One decoding step at full size (B=32, Hq=32, Hkv=8, Nk=16384), plain and with 4
+    chunks, on a row sample of eight heads."""
+    w = workloads.EXTRA_WORKLOADS["decode_b32_h32kv8_q1_k16k_d128"]
+    q, k, v = workloads.make_inputs(w)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    rows = workloads.sample_rows(w, [0], heads=[0, 1, 5, 100, 513, 777, 1000, 1023])
+    ro, rlse = oracle.attention(q, k, v, scale=w.scale, causal=True, rows=rows)
+    rt = torch.from_numpy(rows).to(dev)
+    for splits in (0, 4):
+        o, lse = fa.forward_ext(qd, kd, vd, scale=w.scale, causal=True, num_splits=splits)
+        torch.cuda.synchronize()
+        assert fa.check_status() == 0
+        compare_rows(o.reshape(-1, w.d)[rt].double().cpu().numpy(), lse.reshape(-1)[rt].double().cpu().numpy(),
+                     ro, rlse)
+
