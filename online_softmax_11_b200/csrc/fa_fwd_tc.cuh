@@ -88,8 +88,8 @@ struct Layout {
   static constexpr int kBarKvFull = kBarQEmpty + NQ;      // [kStages]
   static constexpr int kBarKvEmpty = kBarKvFull + kStages;
   static constexpr int kBarSFull = kBarKvEmpty + kStages; // [NQ]
-  static constexpr int kBarPFull = kBarSFull + NQ;        // [NQ]
-  static constexpr int kBarOFull = kBarPFull + NQ;        // [NQ]
+  static constexpr int kBarPFull = kBarSFull + NQ;        // [NQ][2]: P of key half 0 / 1 stored
+  static constexpr int kBarOFull = kBarPFull + 2 * NQ;    // [NQ]
   static constexpr int kBarDrain = kBarOFull + NQ;
   static constexpr int kNumBars = kBarDrain + NQ;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // u32 tmem base, int abort flag
@@ -435,7 +435,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[L::kBarQFull + i], 1);
       mbar_init(&bars[L::kBarQEmpty + i], 1);
       mbar_init(&bars[L::kBarSFull + i], 1);
-      mbar_init(&bars[L::kBarPFull + i], 128);
+      mbar_init(&bars[L::kBarPFull + 2 * i], 128);
+      mbar_init(&bars[L::kBarPFull + 2 * i + 1], 128);
       mbar_init(&bars[L::kBarOFull + i], 1);
     }
     for (int s = 0; s < L::kStages; ++s) {
@@ -564,12 +565,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (n > 0) {
             if (use_pv) {
               if (!mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
-              if (!mbar_wait(&bars[L::kBarPFull + i], p_phase, ctl)) return false;
+              // O_i (+)= P_i V in two halves of 64 keys, each as soon as the softmax has
+              // stored that half of P (the second half of the softmax overlaps the first
+              // half's MMAs): A = 16 keys of P = 8 TMEM columns per step; B = 16 key rows
+              // of V (128 B each); the two 64-column slabs of V are kHalfBytes apart
+              const uint64_t dv = dvring + ((vslot * L::kTileBytes) >> 4);
+              if (!mbar_wait(&bars[L::kBarPFull + 2 * i], p_phase, ctl)) return false;
+              tc_fence_after();
+              mma_ts_kloop4(d_o, d_s, dv, kIdescPV, o_acc);
+              if (!mbar_wait(&bars[L::kBarPFull + 2 * i + 1], p_phase, ctl)) return false;
               p_phase ^= 1u;
               tc_fence_after();
-              // O_i (+)= P_i V: A = 16 keys of P = 8 TMEM columns per step; B = 16 key rows
-              // of V (128 B each); the two 64-column slabs of V are kHalfBytes apart
-              mma_ts_kloop8(d_o, d_s, dvring + ((vslot * L::kTileBytes) >> 4), kIdescPV, o_acc);
+              mma_ts_kloop4(d_o, d_s + 32, dv + 512, kIdescPV, 1u);
               o_acc = 1;
               if (n - 1 == n_last) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
               mma_commit(&bars[L::kBarKvEmpty + vslot]);
@@ -733,6 +740,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             lt += make_p<PMode::kCapGeneral>(s, tp, 0.f, p.cap_inner, p.cap_outer, m_use);
           }
+          // this half of P is in tensor memory: its P.V can start
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&bars[L::kBarPFull + 2 * i + h]);
         }
         if (!p.use_softcap) {
           const float u = fmaf(mx, p.scale_log2, -m_use);
@@ -753,9 +764,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // bf16; that one term dominates peaked rows, the other roundings average out.
         l += lt;
         lr += lt + (__bfloat162float(__float2bfloat16_rn(pmax)) - pmax);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars[L::kBarPFull + i]);
         o_valid = true;
       }
 

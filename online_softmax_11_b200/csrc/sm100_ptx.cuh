@@ -212,6 +212,24 @@ __device__ __forceinline__ void mma_ts_kloop8(uint32_t d_tmem, uint32_t a_tmem, 
       : "memory");
 }
 
+// Half of that K loop: 4 steps (64 keys) from P column a_tmem and V descriptor b_desc.
+__device__ __forceinline__ void mma_ts_kloop4(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred pt, p0;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.eq.u32 pt, 0, 0;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+      "add.u32 a, %1, 8;\n\tadd.s64 b, %2, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
+      "add.u32 a, %1, 16;\n\tadd.s64 b, %2, 256;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
+      "add.u32 a, %1, 24;\n\tadd.s64 b, %2, 384;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05 operation this thread issued so far is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
