@@ -303,12 +303,15 @@ __global__ void __launch_bounds__(kTopkThreads, 2)
     lm = fmaxf(lm, xr[tail0 + tid]);
   }
   int i = tid;
-  for (; i + nt < sp.n4; i += 2 * nt) {  // two loads in flight per thread
-    const float4 v0 = __ldg(x4 + i);
-    const float4 v1 = __ldg(x4 + i + nt);
-    md_add4(s, v0.x, v0.y, v0.z, v0.w);
-    md_add4(s, v1.x, v1.y, v1.z, v1.w);
-    lm = fmaxf(lm, fmaxf(fmaxf(fmaxf(v0.x, v0.y), fmaxf(v0.z, v0.w)), fmaxf(fmaxf(v1.x, v1.y), fmaxf(v1.z, v1.w))));
+  for (; i + 3 * nt < sp.n4; i += 4 * nt) {  // four loads in flight per thread
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = __ldg(x4 + i + u * nt);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      md_add4(s, v[u].x, v[u].y, v[u].z, v[u].w);
+      lm = fmaxf(lm, fmaxf(fmaxf(v[u].x, v[u].y), fmaxf(v[u].z, v[u].w)));
+    }
   }
   for (; i < sp.n4; i += nt) {
     const float4 v = __ldg(x4 + i);
@@ -329,7 +332,23 @@ __global__ void __launch_bounds__(kTopkThreads, 2)
   };
   if (tid < sp.head) keep(xr[tid], tid);
   if (tid < sp.tail) keep(xr[tail0 + tid], tail0 + tid);
-  for (int i = tid; i < sp.n4; i += nt) {
+  int j = tid;
+  for (; j + 3 * nt < sp.n4; j += 4 * nt) {  // four loads in flight per thread
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = __ldcs(x4 + j + u * nt);  // last use of the row
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (fmaxf(fmaxf(v[u].x, v[u].y), fmaxf(v[u].z, v[u].w)) >= tau) {
+        const int c = sp.head + 4 * (j + u * nt);
+        keep(v[u].x, c);
+        keep(v[u].y, c + 1);
+        keep(v[u].z, c + 2);
+        keep(v[u].w, c + 3);
+      }
+    }
+  }
+  for (int i = j; i < sp.n4; i += nt) {
     const float4 v = __ldcs(x4 + i);  // last use of the row
     if (fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)) >= tau) {
       const int c = sp.head + 4 * i;

@@ -40,7 +40,9 @@ def logits(rows, V, seed, scale=4.0):
     return torch.randn((rows, V), generator=g, dtype=torch.float32) * scale
 
 
-SHAPES = [(1, 1), (3, 5), (4, 127), (2, 1000), (5, 4099), (3, 16384), (2, 32000), (2, 50257), (1, 262144)]
+# long rows (up to a million floats: the second read of a row then comes from HBM)
+SHAPES = [(1, 1), (3, 5), (4, 127), (2, 1000), (5, 4099), (3, 16384), (2, 32000), (2, 50257), (2, 65536),
+          (2, 70001), (3, 100003), (1, 262144), (2, 1000000)]
 
 
 @pytest.mark.parametrize("rows,V", SHAPES)
