@@ -349,41 +349,68 @@ def gpu_arm(args, w):
     # ---- e2e: pinned host inputs -> device, forward, outputs -> pinned host, per step
     e2e = None
     if not args.no_e2e:
+        # Every step copies its inputs from pinned host memory, runs the forward through
+        # the public call and copies O and LSE back.  Steps are pipelined over three
+        # streams with two buffer sets: step i's inputs go in while step i-1 computes and
+        # step i-2's outputs come back (the two copy directions and the kernels overlap).
         qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
         op = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
         lp = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bufs = [(torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(o),
+                 torch.empty_like(lse)) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_done = [torch.cuda.Event() for _ in range(2)]
+        comp_done = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
+        used = [False, False]
 
-        def e2e_step():
-            qd.copy_(qp, non_blocking=True)
-            kd.copy_(kp, non_blocking=True)
-            vd.copy_(vp, non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            qd, kd, vd, od, ld = bufs[b]
+            if used[b]:  # the buffers' previous step has finished computing / copying out
+                s_in.wait_event(comp_done[b])
+                stream.wait_event(out_done[b])
+            with torch.cuda.stream(s_in):
+                qd.copy_(qp, non_blocking=True)
+                kd.copy_(kp, non_blocking=True)
+                vd.copy_(vp, non_blocking=True)
+                in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
             if general:
-                launch(qd, kd, vd, o, lse)
+                launch(qd, kd, vd, od, ld)
             else:
-                fa.forward(qd, kd, vd, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, out=o,
-                           lse=lse, stream=stream)
-            op.copy_(o, non_blocking=True)
-            lp.copy_(lse, non_blocking=True)
+                fa.forward(qd, kd, vd, scale=w.scale, causal=w.causal, window=w.window, softcap=w.softcap, out=od,
+                           lse=ld, stream=stream)
+            comp_done[b].record(stream)
+            s_out.wait_event(comp_done[b])
+            with torch.cuda.stream(s_out):
+                op.copy_(od, non_blocking=True)
+                lp.copy_(ld, non_blocking=True)
+                out_done[b].record(s_out)
+            used[b] = True
 
-        e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize(dev)
         if ws > 1:
             dist.barrier()
         n_e2e = max(1, min(args.e2e_steps, args.steps))
         es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        es.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        ee.record(stream)
+        es.record(s_in)
+        for i in range(n_e2e):
+            e2e_step(i)
+        s_out.wait_event(comp_done[(n_e2e - 1) % 2])
+        ee.record(s_out)
         torch.cuda.synchronize(dev)
         te_ms = max_over_ranks(es.elapsed_time(ee), dev)
         h2d = (q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size())
         d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
         e2e = {"value": job_tflops(ws, flop_per_step, n_e2e, te_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "ms_per_step": te_ms / n_e2e}
-        del qp, kp, vp, op, lp, qd, kd, vd
+               "ms_per_step": te_ms / n_e2e, "pipelined": "copies in, kernel, copies out on three streams"}
+        if fa.check_status() != 0:
+            raise RuntimeError("device status word set during the end-to-end run")
+        del qp, kp, vp, op, lp, bufs
 
     # ---- CPU baseline: the fp64 oracle on a bounded row sample (rank 0, N = 1 only)
     cpu = None
@@ -542,33 +569,65 @@ def softmax_arm(args, sw):
 
     e2e = None
     if not args.no_e2e:
+        # pinned input copied in, the kernel, outputs copied back, every step; steps are
+        # pipelined over three streams with two buffer sets (as in the attention arm)
         xp = x_h.pin_memory()
         outp = torch.empty(y.shape if op == "softmax" else probs.shape, dtype=torch.float32, pin_memory=True)
         ip = torch.empty(idx.shape, dtype=torch.int32, pin_memory=True)
-        xd = torch.empty_like(x)
+        bufs = [(torch.empty_like(x), torch.empty_like(y) if op == "softmax" else None, torch.empty_like(probs),
+                 torch.empty_like(idx), torch.empty_like(lse)) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_done = [torch.cuda.Event() for _ in range(2)]
+        comp_done = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
+        used = [False, False]
 
-        def e2e_step():
-            xd.copy_(xp, non_blocking=True)
-            step(xd)
+        def e2e_step(i):
+            b = i % 2
+            xd, yd, pd, idd, ld = bufs[b]
+            if used[b]:
+                s_in.wait_event(comp_done[b])
+                stream.wait_event(out_done[b])
+            with torch.cuda.stream(s_in):
+                xd.copy_(xp, non_blocking=True)
+                in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
             if op == "softmax":
-                outp.copy_(y, non_blocking=True)
+                rc = lib.fa_softmax(xd.data_ptr(), yd.data_ptr(), ld.data_ptr(), sw.rows, sw.V, sh)
             else:
-                outp.copy_(probs, non_blocking=True)
-                ip.copy_(idx, non_blocking=True)
+                rc = lib.fa_softmax_topk(xd.data_ptr(), pd.data_ptr(), idd.data_ptr(), ld.data_ptr(), sw.rows, sw.V,
+                                         sw.k, sh)
+            if rc != 0:
+                raise fa.FAError(rc, lib, "fa_" + op)
+            comp_done[b].record(stream)
+            s_out.wait_event(comp_done[b])
+            with torch.cuda.stream(s_out):
+                if op == "softmax":
+                    outp.copy_(yd, non_blocking=True)
+                else:
+                    outp.copy_(pd, non_blocking=True)
+                    ip.copy_(idd, non_blocking=True)
+                out_done[b].record(s_out)
+            used[b] = True
 
-        e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize(dev)
+        if ws > 1:
+            dist.barrier()
         n_e2e = max(1, min(args.e2e_steps, args.steps))
         es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        es.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        ee.record(stream)
+        es.record(s_in)
+        for i in range(n_e2e):
+            e2e_step(i)
+        ee.record(s_out)
         torch.cuda.synchronize(dev)
         te = max_over_ranks(es.elapsed_time(ee), dev)
         d2h = y.numel() * 4 if op == "softmax" else probs.numel() * 4 + idx.numel() * 4
         e2e = {"value": ws * nbytes * n_e2e / (te / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": x.numel() * 4,
-               "d2h_bytes_per_step": d2h, "steps": n_e2e, "ms_per_step": te / n_e2e}
+               "d2h_bytes_per_step": d2h, "steps": n_e2e, "ms_per_step": te / n_e2e,
+               "pipelined": "copies in, kernel, copies out on three streams"}
+        del xp, outp, ip, bufs
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
