@@ -427,7 +427,8 @@ def gpu_arm(args, w):
         kernel = f"fa_decode_kernel<{w.d}>"
     else:
         kernel = (f"fa_fwd_tc_kernel<{w.d}, {'true' if args.splits > 0 else 'false'}, "
-                  f"{'true' if (w.n_sink > 0 and w.window > 0) else 'false'}>")
+                  f"{'true' if (w.n_sink > 0 and w.window > 0) else 'false'}, "
+                  f"{'true' if w.softcap > 0 else 'false'}>")
     # algorithmic bytes: Q, K, V read once, O and LSE written once
     alg_bytes = float(q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size()
                       + o.numel() * o.element_size() + lse.numel() * lse.element_size())

@@ -47,26 +47,33 @@ int current_device(int* dev) {
 
 template <int D, bool kSplit, bool kSinks>
 cudaError_t set_tc_smem() {
-  return cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              fa::tc::Layout<D>::kSmemLaunch);
+  cudaError_t e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, fa::tc::Layout<D>::kSmemLaunch);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, fa::tc::Layout<D>::kSmemLaunch);
+  return e;
 }
 
 template <int D, bool kSplit, bool kSinks>
-void launch_tc_kernel(unsigned grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+void launch_tc_kernel(bool cap, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const fa::tc::Params& p, cudaStream_t s) {
-  fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks><<<grid, fa::tc::kThreads, fa::tc::Layout<D>::kSmemLaunch, s>>>(mq, mk, mv,
-                                                                                                            p);
+  constexpr int kSmem = fa::tc::Layout<D>::kSmemLaunch;
+  if (cap)
+    fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, true><<<grid, fa::tc::kThreads, kSmem, s>>>(mq, mk, mv, p);
+  else
+    fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, false><<<grid, fa::tc::kThreads, kSmem, s>>>(mq, mk, mv, p);
 }
 
 template <int D>
-void launch_tc_variant(bool split, bool sinks, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mk,
+void launch_tc_variant(bool split, bool sinks, bool cap, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mk,
                        const CUtensorMap& mv, const fa::tc::Params& p, cudaStream_t s) {
   if (split) {
-    if (sinks) launch_tc_kernel<D, true, true>(grid, mq, mk, mv, p, s);
-    else launch_tc_kernel<D, true, false>(grid, mq, mk, mv, p, s);
+    if (sinks) launch_tc_kernel<D, true, true>(cap, grid, mq, mk, mv, p, s);
+    else launch_tc_kernel<D, true, false>(cap, grid, mq, mk, mv, p, s);
   } else {
-    if (sinks) launch_tc_kernel<D, false, true>(grid, mq, mk, mv, p, s);
-    else launch_tc_kernel<D, false, false>(grid, mq, mk, mv, p, s);
+    if (sinks) launch_tc_kernel<D, false, true>(cap, grid, mq, mk, mv, p, s);
+    else launch_tc_kernel<D, false, false>(cap, grid, mq, mk, mv, p, s);
   }
 }
 
@@ -326,10 +333,11 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   // persistent: one CTA per SM (never more CTAs than units)
   const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
   const bool sinks = p.n_sink > 0;
+  const bool cap = p.use_softcap != 0;
   if (d == 128)
-    launch_tc_variant<128>(split, sinks, grid, mq, mk, mv, p, s);
+    launch_tc_variant<128>(split, sinks, cap, grid, mq, mk, mv, p, s);
   else
-    launch_tc_variant<64>(split, sinks, grid, mq, mk, mv, p, s);
+    launch_tc_variant<64>(split, sinks, cap, grid, mq, mk, mv, p, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   if (split) {

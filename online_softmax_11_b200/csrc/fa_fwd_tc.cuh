@@ -414,7 +414,9 @@ __device__ __forceinline__ void for_each_tile(const Params& p, F&& f) {
 // kSinks: the launch has attention sinks (a separate run of sink tiles may precede the
 // window's tiles); without them every key-tile set is one run and the loops are the
 // plain ranges.
-template <int D, bool kSplit, bool kSinks>
+// kCap: logit soft-cap on; without it the soft-cap code is not compiled in (fewer live
+// registers in the softmax).
+template <int D, bool kSplit, bool kSinks, bool kCap>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -672,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
             mx_emu = fmax3(mx_emu, s[c + 6], s[c + 7]);
           }
-          if (p.use_softcap) {
+          if constexpr (kCap) {
 #pragma unroll
             for (int c = 0; c < kHalf; c += 4) {
               mn0 = fmin3(mn0, s[c], s[c + 1]);
@@ -683,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx_emu));
         const float mn = fminf(mn0, mn1);
         float m_tile;
-        if (p.use_softcap)
+        if constexpr (kCap)
           m_tile = (mx == -CUDART_INF_F) ? -CUDART_INF_F : p.cap_outer * tanh_cap(mx * p.cap_inner);
         else
           m_tile = mx * p.scale_log2;
@@ -718,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the same instructions as in make_p (so it is bit-identical to the value packed).
         float lt = 0.f, pmax;
         int wtier = 0;
-        if (p.use_softcap) {
+        if constexpr (kCap) {
           const float amax = fmaxf(fabsf(mx), fabsf(mn)) * p.cap_inner;  // max |x| of the row
           const int tier = need_mask ? 2 : (amax < 0.12f ? 0 : (amax < 0.3f ? 1 : 2));
           wtier = __reduce_max_sync(0xffffffffu, tier);
@@ -728,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float s[kHalf];
           load_half<kSinks>(lane_base + colS + h * kHalf, h * kHalf, need_mask, sink_cols, h_lo, h_hi, c_hi, s);
           const uint32_t tp = lane_base + colS + h * (kHalf / 2);
-          if (!p.use_softcap) {
+          if constexpr (!kCap) {
             if (need_mask)
               lt += make_p<PMode::kPlainMufu>(s, tp, p.scale_log2, 0.f, 0.f, m_use);
             else
@@ -745,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(&bars[L::kBarPFull + 2 * i + h]);
         }
-        if (!p.use_softcap) {
+        if constexpr (!kCap) {
           const float u = fmaf(mx, p.scale_log2, -m_use);
           pmax = (!need_mask && mx_emu == mx) ? exp2_fma_pair(make_float2(u, u)).x : ex2_approx(u);
         } else {
