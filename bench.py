@@ -639,7 +639,8 @@ def softmax_arm(args, sw):
     peak_bw = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     achieved = nbytes / (per_launch / 1e3) / 1e9
     kmax = next(c for c in (4, 8, 16, 32) if sw.k <= c)
-    kernel = "softmax_online_kernel" if op == "softmax" else f"softmax_topk_kernel<{kmax}>"
+    kernel = ("softmax_online_kernel" if op == "softmax" else
+              f"softmax_topk_kernel<{kmax}, {512 if sw.V <= 131072 else 1024}>")
     if rank == 0:
         emit({"metric": SOFTMAX_METRIC[op], "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
               "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,

@@ -587,6 +587,26 @@ int fa_softmax(const float* x, float* y, float* lse, int rows, int V, void* stre
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
+}  // extern "C"
+
+namespace {
+
+template <int T>
+void launch_topk(unsigned g, const float* x, float* probs, int* idx, float* lse, int V, int K, cudaStream_t s) {
+  if (K <= 4)
+    fa::smx::softmax_topk_kernel<4, T><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
+  else if (K <= 8)
+    fa::smx::softmax_topk_kernel<8, T><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
+  else if (K <= 16)
+    fa::smx::softmax_topk_kernel<16, T><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
+  else
+    fa::smx::softmax_topk_kernel<32, T><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
+}
+
+}  // namespace
+
+extern "C" {
+
 int fa_softmax_topk(const float* x, float* probs, int* idx, float* lse, int rows, int V, int K, void* stream) {
   if (rows < 0 || V < 0) return FA_ERR_BAD_SHAPE;
   if (K < 1 || K > fa::smx::kMaxTopK || (rows > 0 && K > V)) return FA_ERR_BAD_ARG;
@@ -598,15 +618,10 @@ int fa_softmax_topk(const float* x, float* probs, int* idx, float* lse, int rows
   if ((rc = prepare_device(dev)) != FA_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned g = static_cast<unsigned>(rows);
-  constexpr int T = fa::smx::kTopkThreads;
-  if (K <= 4)
-    fa::smx::softmax_topk_kernel<4><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
-  else if (K <= 8)
-    fa::smx::softmax_topk_kernel<8><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
-  else if (K <= 16)
-    fa::smx::softmax_topk_kernel<16><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
+  if (V <= 131072)
+    launch_topk<fa::smx::kTopkThreadsShort>(g, x, probs, idx, lse, V, K, s);
   else
-    fa::smx::softmax_topk_kernel<32><<<g, T, 0, s>>>(x, probs, idx, lse, V, K);
+    launch_topk<fa::smx::kTopkThreadsLong>(g, x, probs, idx, lse, V, K, s);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }

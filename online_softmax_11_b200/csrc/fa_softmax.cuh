@@ -29,7 +29,11 @@ namespace fa {
 namespace smx {
 
 constexpr int kSoftmaxThreads = 1024;
-constexpr int kTopkThreads = 1024;
+// top-K blocks: 512 threads (four blocks, four rows in flight per SM) up to rows of 128 K
+// floats, 1024 threads (two per SM) for longer rows, where fewer, larger blocks measured
+// faster
+constexpr int kTopkThreadsShort = 512;
+constexpr int kTopkThreadsLong = 1024;
 constexpr int kMaxTopK = 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -274,8 +278,8 @@ __device__ __forceinline__ float block_kth_bound(float lm, int K, float* red_f) 
 // row with a per-thread list of the KMAX best.
 constexpr int kCand = 1024;
 
-template <int KMAX>
-__global__ void __launch_bounds__(kTopkThreads, 2)
+template <int KMAX, int kTopkThreads>
+__global__ void __launch_bounds__(kTopkThreads, 2048 / kTopkThreads)
     softmax_topk_kernel(const float* __restrict__ x, float* __restrict__ probs, int* __restrict__ idx,
                         float* __restrict__ lse, int V, int K) {
   __shared__ MD red[32];
