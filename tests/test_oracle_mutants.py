@@ -8,7 +8,6 @@ mistakes live only in these temporary copies, on the CPU.
 import functools
 import os
 import subprocess
-import tempfile
 
 import pytest
 
@@ -47,14 +46,18 @@ MUTANTS = {
 }
 
 
-@functools.lru_cache(maxsize=None)
-def _build_mutant(name):
+@pytest.fixture(scope="module")
+def mutant_dir(tmp_path_factory):
+    """One pytest-managed temporary directory for the mutant builds of this module."""
+    return str(tmp_path_factory.mktemp("oracle_mutants"))
+
+
+def _build_mutant(name, directory):
     old, new = MUTANTS[name]
     src = open(SRC).read()
     assert src.count(old) == 1, f"mutation site for {name} not unique"
-    tmp = tempfile.mkdtemp(prefix="oracle_mutant_")
-    c_path = os.path.join(tmp, "attn.c")
-    so_path = os.path.join(tmp, "libattn.so")
+    c_path = os.path.join(directory, f"{name}.c")
+    so_path = os.path.join(directory, f"lib{name}.so")
     open(c_path, "w").write(src.replace(old, new))
     subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-pthread", c_path, "-o", so_path, "-lm"],
                    check=True)
@@ -62,8 +65,8 @@ def _build_mutant(name):
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_planted_mistake_fails_a_pin(name):
-    lib = _build_mutant(name)
+def test_planted_mistake_fails_a_pin(name, mutant_dir):
+    lib = _build_mutant(name, mutant_dir)
     attn = functools.partial(oracle.attention, _lib=lib)
     failed = pin_suite.failures(attn)
     assert failed, f"planted mistake {name!r} passed every pin"
