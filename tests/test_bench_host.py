@@ -1,0 +1,42 @@
+"""Host-side arithmetic of the benchmark (no GPU): the FLOP and byte counts it divides by."""
+import numpy as np
+
+import bench
+import oracle
+import workloads
+from tests.pin_suite import _kept_keys
+
+
+def test_kept_keys_per_row_matches_brute_force():
+    """4 d FLOPs per kept pair: the per-row key counts of the general workloads equal the
+    key sets built from the mask's words (queries at the last Nq positions, window,
+    sinks, causal)."""
+    for (N, nq, W, S, causal) in [(50, 0, 7, 3, True), (50, 10, 7, 3, True), (40, 55, 5, 2, True),
+                                  (30, 0, 0, 0, False), (30, 12, 0, 0, False), (64, 0, 1, 4, True),
+                                  (64, 0, 10, 30, True), (300, 1, 0, 0, True)]:
+        w = workloads.Workload("t", 0, 1, 1, 1, N, 8, "bfloat16", causal, W, 0.0, nq=nq, n_sink=S)
+        got = bench.kept_keys_per_row(w, np.arange(w.Nq))
+        want = [len(_kept_keys(i + N - w.Nq, N, causal, W, S)) for i in range(w.Nq)]
+        assert list(got) == want, (N, nq, W, S)
+
+
+def test_closed_flops_follow_the_convention():
+    for n in (2, 3, 4, 5):
+        w = workloads.BY_NUMBER[n]
+        assert bench.closed_flops(w) == oracle.flops(w.B, w.Hq, w.N, w.d, w.causal, w.window, convention="closed")
+    # the general workloads count kept pairs exactly
+    w = workloads.EXTRA_WORKLOADS["decode_b32_h32kv8_q1_k16k_d128"]
+    assert bench.closed_flops(w) == 4.0 * w.d * w.B * w.Hq * w.N
+    w = workloads.EXTRA_WORKLOADS["chunk_b4_h32kv8_q1k_k16k_d128"]
+    pairs = w.Nq * (w.N - w.Nq) + w.Nq * (w.Nq + 1) // 2
+    assert bench.closed_flops(w) == 4.0 * w.d * w.B * w.Hq * pairs
+
+
+def test_softmax_bytes():
+    sw = workloads.SOFTMAX_WORKLOADS["softmax_r4k_v32k"]
+    assert bench.softmax_bytes(sw, "softmax") == sw.rows * sw.V * 8 + sw.rows * 4
+    assert bench.softmax_bytes(sw, "softmax_topk") == sw.rows * sw.V * 4 + sw.rows * sw.k * 8 + sw.rows * 4
+
+
+def test_job_throughput_is_the_whole_job_over_the_slowest_rank():
+    assert bench.job_tflops(4, 1e12, 10, 1000.0) == 4 * 1e12 * 10 / 1.0 / 1e12
