@@ -49,6 +49,7 @@ import workloads  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s on 1 B200 and % of dense BF16 tensor peak"
 UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024  # B200 L2 (126 MB)
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 KERNEL_SOURCES = ["online_softmax_11_b200/csrc/fa_fwd_tc.cuh", "online_softmax_11_b200/csrc/sm100_ptx.cuh",
                   "online_softmax_11_b200/csrc/fa_api.cu"]
@@ -327,16 +328,32 @@ def gpu_arm(args, w):
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    in_bytes = q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size()
+    small = in_bytes < L2_BYTES
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(args.steps):
-        step()
-    end.record(stream)
-    torch.cuda.synchronize(dev)
+    if not small:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        elapsed_ms = start.elapsed_time(end)
+    else:
+        # inputs that fit in L2: flush it (write a larger buffer) before every step and
+        # time each step alone with its own events
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        elapsed_ms = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            start.record(stream)
+            step()
+            end.record(stream)
+            end.synchronize()
+            elapsed_ms += start.elapsed_time(end)
+        del flush
     if ws > 1:
         dist.barrier()
-    elapsed_ms = start.elapsed_time(end)
     clocks = sampler.stop() if sampler is not None else None
     if fa.check_status() != 0:
         raise RuntimeError("device status word set during the timed region")
@@ -423,7 +440,9 @@ def gpu_arm(args, w):
     peaks, peaks_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_bw = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    if (w.Hq // w.Hkv) * w.Nq <= 16:  # the group's query rows fit one 16-row block
+    if w.dtype == "float32":  # the fp32 CUDA-core path
+        kernel = f"fa_fwd_f32_kernel<{(w.d + 31) // 32}>"
+    elif (w.Hq // w.Hkv) * w.Nq <= 16:  # the group's query rows fit one 16-row block
         kernel = f"fa_decode_kernel<{w.d}>"
     else:
         kernel = (f"fa_fwd_tc_kernel<{w.d}, {'true' if args.splits > 0 else 'false'}, "
@@ -432,7 +451,18 @@ def gpu_arm(args, w):
     # algorithmic bytes: Q, K, V read once, O and LSE written once
     alg_bytes = float(q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size()
                       + o.numel() * o.element_size() + lse.numel() * lse.element_size())
-    if flop_per_step / alg_bytes >= peak * 1e12 / (peak_bw * 1e9):
+    if w.dtype == "float32":
+        # plain FP32 FMA arithmetic: peak = SMs x 128 FP32 lanes x 2 flop x the SM clock
+        # seen (1965 MHz when no sample was taken)
+        sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
+        peak_alu = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
+        achieved = flop_per_step / (per_launch_ms / 1e3) / 1e12
+        roofline = {"bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": UNIT,
+                    "frac": achieved / peak_alu, "traffic": None,
+                    "peak_source": "SMs x 128 FP32 lanes x 2 flop x SM clock (derived, no tensor cores)",
+                    "kernel": kernel, "algorithmic_flop_per_launch": flop_per_step,
+                    "note": "n = 64, d = 32: one launch of a few microseconds, bound by launch latency"}
+    elif flop_per_step / alg_bytes >= peak * 1e12 / (peak_bw * 1e9):
         achieved = flop_per_step / (per_launch_ms / 1e3) / 1e12
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
                     "traffic": load_traffic(w.name), "peak_source": f"bf16_tflops (burst) of {peaks_src}",
@@ -449,13 +479,16 @@ def gpu_arm(args, w):
         cfg = {"workload": w.name, **{k: v for k, v in w.describe().items() if k != "workload"},
                "flop_convention": ("4 d per kept (query, key) pair" if (w.nq > 0 or w.n_sink > 0) else
                                    "4 B Hq N^2 d, /2 causal; 4 B Hq d (N W - W^2/2) with a window"),
-               "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{ws} (independent batches)"}
+               "l2": ("L2 flushed before every step (inputs smaller than L2); steps timed one by one" if small
+                      else "inputs larger than L2 (no flush needed)"),
+               "parallelism": f"replicas x{ws} (independent batches)"}
         if args.splits > 0:
             cfg["split_kv"] = args.splits
         emit({
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32" if w.dtype == "float32" else "bf16",
+            "data": "synthetic", "config": cfg,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": args.steps * (2 if args.splits > 0 else 1),
         })
@@ -689,8 +722,6 @@ def main(argv=None):
     if args.workload in workloads.SOFTMAX_WORKLOADS:
         ap.error("softmax workloads need --op softmax or --op softmax_topk")
     w = workloads.ALL_WORKLOADS[args.workload or workloads.HEADLINE]
-    if w.dtype != "bfloat16" and args.impl == "ours":
-        ap.error("the benchmark times the bf16 tensor-core path")
     if args.batch is not None:
         w = w.with_(B=args.batch)
     if args.impl == "reference":
