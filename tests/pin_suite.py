@@ -411,6 +411,50 @@ def pin_cross_attention(attn):
     assert np.array_equal(o[0, 0, 3:], ref[0, 0]) and np.array_equal(lse[0, 0, 3:], rl[0, 0])
 
 
+def _bf16_from_bits(bits):
+    """bf16 torch tensor whose elements have exactly the given 16-bit patterns."""
+    b = np.ascontiguousarray(np.asarray(bits, dtype=np.uint16))
+    return torch.from_numpy(b.view(np.int16).copy()).view(torch.bfloat16)
+
+
+def pin_bf16_inputs(attn):
+    """bf16 inputs are read as the exact values they store: the oracle on bf16 tensors
+    equals, bit for bit, the oracle on the same tensors widened to float64 by torch
+    (an independent library conversion).  The values cover both signs, bf16
+    subnormals (a query row of subnormals against keys of 2^120 makes them decide the
+    scores) and magnitudes up to 2^120 (a one-hot softmax copies such a V row into O),
+    so a wrong shift, a byte swap or a lost sign changes the output.  MHA, GQA and
+    cross shapes, with the masks and the soft-cap."""
+    rng = _rng(97)
+
+    def rand_bits(shape):
+        x = torch.from_numpy(rng.standard_normal(shape).astype(np.float32)).to(torch.bfloat16)
+        return x.view(torch.int16).numpy().view(np.uint16).copy()
+
+    cases = [  # B, Hq, Hkv, Nq, Nk, d, causal, window, cap
+        (1, 2, 2, 7, 7, 5, False, 0, 0.0),
+        (2, 4, 2, 9, 9, 6, True, 0, 0.0),
+        (1, 2, 1, 3, 8, 4, True, 3, 0.0),
+        (1, 2, 2, 6, 6, 4, True, 0, 2.5),
+    ]
+    for B, Hq, Hkv, Nq, Nk, d, causal, window, cap in cases:
+        qb, kb, vb = rand_bits((B, Hq, Nq, d)), rand_bits((B, Hkv, Nk, d)), rand_bits((B, Hkv, Nk, d))
+        # query row 0 of head 0: bf16 subnormals (exponent field 0) of both signs;
+        # key row 0: +-2^120 (0x7b80 / 0xfb80), so q.k of that pair is of order 2^-10
+        qb[0, 0, 0, :] = np.array([0x0001, 0x8003, 0x007F, 0x0040, 0x8011, 0x0002][:d], dtype=np.uint16)
+        kb[0, 0, 0, :] = np.array([0x7B80, 0xFB80, 0x7B80, 0x7B80, 0xFB80, 0x7B80][:d], dtype=np.uint16)
+        # value rows with 2^100 (0x7180), -1.25 * 2^110 (0xf6a0), subnormals, small
+        # negatives and the largest finite bf16 of both signs (0x7f7f / 0xff7f)
+        vb[0, 0, 1, :] = np.array([0x7180, 0xF6A0, 0x0005, 0x8005, 0xBF40, 0x3F81][:d], dtype=np.uint16)
+        vb[0, -1, -1, :] = np.array([0x8001, 0x0080, 0xC2F7, 0x42F7, 0x7F7F, 0xFF7F][:d], dtype=np.uint16)
+        q, k, v = _bf16_from_bits(qb), _bf16_from_bits(kb), _bf16_from_bits(vb)
+        o_b, l_b = attn(q, k, v, scale=0.37, causal=causal, window=window, softcap=cap)
+        o_d, l_d = attn(q.to(torch.float64), k.to(torch.float64), v.to(torch.float64), scale=0.37, causal=causal,
+                        window=window, softcap=cap)
+        assert np.array_equal(o_b, o_d, equal_nan=True) and np.array_equal(l_b, l_d, equal_nan=True)
+        assert np.all(np.isfinite(l_b)) or causal
+
+
 def pin_empty(attn):
     """No queries (or a zero batch) gives empty outputs and no error (oxios returns an
     empty result for empty input)."""

@@ -43,6 +43,12 @@ MUTANTS = {
     "sinks_without_window": ("if (J->window > 0 && pos - j >= J->window && j >= J->n_sink)",
                              "if ((J->window > 0 && pos - j >= J->window) || (J->n_sink > 0 && j >= J->n_sink))"),
     "cross_top_left_causal": ("const int64_t pos = i + (N - Nq);", "const int64_t pos = i;"),
+    # widening of the stored bf16 bits (the top half of an IEEE binary32)
+    "bf16_shift_by_15": ("((const uint16_t*)base)[idx] << 16;", "((const uint16_t*)base)[idx] << 15;"),
+    "bf16_low_half": ("((const uint16_t*)base)[idx] << 16;", "((const uint16_t*)base)[idx];"),
+    "bf16_byte_swap": ("((const uint16_t*)base)[idx] << 16;",
+                       "(uint16_t)((((const uint16_t*)base)[idx] >> 8) | (((const uint16_t*)base)[idx] << 8)) << 16;"),
+    "bf16_sign_dropped": ("((const uint16_t*)base)[idx] << 16;", "(((const uint16_t*)base)[idx] & 0x7FFFu) << 16;"),
 }
 
 
@@ -70,3 +76,22 @@ def test_planted_mistake_fails_a_pin(name, mutant_dir):
     attn = functools.partial(oracle.attention, _lib=lib)
     failed = pin_suite.failures(attn)
     assert failed, f"planted mistake {name!r} passed every pin"
+
+
+def test_bf16_marshalling_mistake_fails_a_pin(monkeypatch):
+    """The Python side hands bf16 tensors to the C oracle as raw 16-bit patterns; handing
+    over the fp16 patterns of the same values instead (a plausible slip) must fail."""
+    import numpy as np
+    import torch
+
+    real = oracle._as_host_array
+
+    def fp16_bits(t):
+        if isinstance(t, torch.Tensor) and t.dtype == torch.bfloat16:
+            h = t.detach().cpu().contiguous().to(torch.float16)
+            return h.view(torch.int16).numpy().view(np.uint16), oracle.DTYPE_CODES["bfloat16"]
+        return real(t)
+
+    monkeypatch.setattr(oracle, "_as_host_array", fp16_bits)
+    with pytest.raises(AssertionError):
+        pin_suite.pin_bf16_inputs(oracle.attention)
