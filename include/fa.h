@@ -216,6 +216,12 @@ int fa_softmax_topk(const float* x, float* probs, int* idx, float* lse, int rows
  * word that kernels of this library set when one of their bounded waits ran out
  * (FA_ERR_TIMEOUT) on the current device, or a pending CUDA error (FA_ERR_CUDA).
  * Returns FA_OK when neither happened.
+ * The status word is ONE word per device, shared by every stream and every caller of
+ * the library on that device: a timeout raised by a kernel on another stream is
+ * reported (and cleared) by whichever fa_check_status call reads the word first, and a
+ * kernel on another stream that is still running when this call returns may set it
+ * afterwards.  Callers that issue work from several streams and need to know which of
+ * them timed out should synchronise all of them (or the device) before checking.
  */
 int fa_check_status(void* stream);
 

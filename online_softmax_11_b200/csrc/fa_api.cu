@@ -6,7 +6,6 @@
 
 #include <cmath>
 #include <cstdint>
-#include <mutex>
 
 #include "fa.h"
 #include "fa_decode.cuh"
@@ -14,6 +13,7 @@
 #include "fa_fwd_tc.cuh"
 #include "fa_merge.cuh"
 #include "fa_softmax.cuh"
+#include "host_once.h"
 
 namespace {
 
@@ -30,10 +30,10 @@ constexpr unsigned long long kWaitLimitNs = 2ull * 1000 * 1000 * 1000;
 
 constexpr int kMaxDevices = 64;
 
-// Per-device facts checked once: compute capability and kernel attributes.
+// Per-device facts checked once: compute capability and kernel attributes (a failed
+// check is retried by the next call, see host_once.h).
 struct DeviceState {
-  std::once_flag once;
-  int status = FA_OK;
+  fa::OnceOnSuccess once;
   int num_sms = 0;
 };
 DeviceState g_dev[kMaxDevices];
@@ -79,18 +79,11 @@ void launch_tc_variant(bool split, bool sinks, bool cap, unsigned grid, const CU
 
 int prepare_device(int dev, int* num_sms = nullptr) {
   DeviceState& st = g_dev[dev];
-  std::call_once(st.once, [&] {
+  const int status = st.once.run([&]() -> int {
     cudaDeviceProp prop;
     cudaError_t e = cudaGetDeviceProperties(&prop, dev);
-    if (e != cudaSuccess) {
-      st.status = cuda_fail(e);
-      return;
-    }
-    if (prop.major != 10 || prop.minor != 0) {  // built for sm_100a only
-      st.status = FA_ERR_UNSUPPORTED;
-      return;
-    }
-    st.num_sms = prop.multiProcessorCount;
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (prop.major != 10 || prop.minor != 0) return FA_ERR_UNSUPPORTED;  // built for sm_100a only
 
     e = cudaFuncSetAttribute(fa::dec::fa_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fa::dec::Smem<128>::kAlloc);
@@ -117,10 +110,12 @@ int prepare_device(int dev, int* num_sms = nullptr) {
       e = cudaFuncSetAttribute(fa::fa_fwd_f32_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, f32_smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(fa::fa_fwd_f32_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, f32_smem);
-    if (e != cudaSuccess) st.status = cuda_fail(e);
+    if (e != cudaSuccess) return cuda_fail(e);
+    st.num_sms = prop.multiProcessorCount;
+    return FA_OK;
   });
   if (num_sms) *num_sms = st.num_sms;
-  return st.status;
+  return status;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda).
@@ -461,27 +456,25 @@ namespace {
 static __device__ __align__(256) unsigned char g_splitkv_scratch[FA_STATIC_SCRATCH_BYTES];
 
 struct ScratchState {
-  std::once_flag once;
-  int status = FA_OK;
+  fa::OnceOnSuccess once;
   void* ptr = nullptr;
 };
 ScratchState g_scratch[kMaxDevices];
 
 // Device address of the scratch array on device `dev` (the current device): looked up
-// once per device, on the first call made with that device current.
+// on the first call made with that device current, and again on later calls until a
+// lookup succeeds (a failed first lookup does not disable the device for good).
 int scratch_address(int dev, void** out) {
   ScratchState& st = g_scratch[dev];
-  std::call_once(st.once, [&] {
+  const int status = st.once.run([&]() -> int {
     void* ptr = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&ptr, g_splitkv_scratch);
-    if (e != cudaSuccess) {
-      st.status = cuda_fail(e);
-      return;
-    }
+    if (e != cudaSuccess) return cuda_fail(e);
     st.ptr = ptr;
+    return FA_OK;
   });
   *out = st.ptr;
-  return st.status;
+  return status;
 }
 
 }  // namespace
