@@ -88,6 +88,15 @@ def load_traffic(workload: str):
     return rec.get("dram_bytes_per_launch")
 
 
+def l2_flush_needed(q, k, v) -> bool:
+    """Flush L2 before every step unless every input is re-read from HBM anyway.  The
+    decision is taken on Q + K + V and, separately, on K + V: with grouped-query
+    attention K and V can fit in L2 while Q does not, and K / V tiles left in L2 by one
+    launch would then be read warm by the next."""
+    nbytes = [t.numel() * t.element_size() for t in (q, k, v)]
+    return sum(nbytes) < L2_BYTES or nbytes[1] + nbytes[2] < L2_BYTES
+
+
 def kept_keys_per_row(w, i):
     """Keys each query row i (numpy array) keeps: positions p = i + N - Nq, keys up to p
     (causal), the window's most recent ones plus the sinks below it."""
@@ -114,48 +123,126 @@ def closed_flops(w) -> float:
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """SM clock, power and clock-event reasons sampled while the timed region runs.
+
+    A background thread reads NVML every ``period_ms`` (read-only queries: current and
+    maximum SM clock, power draw, active clock-event reasons); ``nvidia-smi -lms`` is the
+    fallback when the NVML binding is missing.  Only samples taken between
+    ``mark_start()`` and ``mark_end()`` (host times around the timed region, which ends
+    with a device synchronisation) are reported.  The GPU is found by the UUID of the
+    CUDA device, so a CUDA_VISIBLE_DEVICES remapping cannot point NVML at another GPU.
+    """
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int, period_ms: int = 50):
+    def __init__(self, device, period_ms: float = 2.0):
+        import threading
+        self.samples = []  # (host time, sm MHz, max sm MHz, power W, set of reason names)
+        self.t0 = self.t1 = None
         self.proc = None
+        self.thread = None
+        self.source = None
+        self._stop = threading.Event()
+        handle = self._nvml_handle(device)
+        if handle is not None:
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll_nvml, args=(handle, period_ms / 1e3), daemon=True)
+            self.thread.start()
+            return
         try:
+            import torch
+            index = device.index if isinstance(device, torch.device) and device.index is not None else 0
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", str(period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "10"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi"
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
+            self.thread.start()
         except OSError:
             self.proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
+    @staticmethod
+    def _nvml_handle(device):
         try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device)
+            uuid = str(getattr(props, "uuid", ""))
+            if uuid:
+                try:
+                    return pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+                except pynvml.NVMLError:
+                    pass
+            if os.environ.get("CUDA_VISIBLE_DEVICES") is None:
+                return pynvml.nvmlDeviceGetHandleByIndex(torch.device(device).index or 0)
+        except Exception:  # noqa: BLE001 - no NVML: fall back to nvidia-smi
+            return None
+        return None
+
+    def _poll_nvml(self, handle, period_s):
+        import pynvml
+        bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+        smax = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
+        while not self._stop.is_set():
+            t = time.perf_counter()
+            try:
+                sm = float(pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM))
+                mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                power = pynvml.nvmlDeviceGetPowerUsage(handle) / 1e3
+            except pynvml.NVMLError:
+                break
+            self.samples.append((t, sm, smax, power, {n for n, b in bits.items() if mask & b}))
+            time.sleep(period_s)
+
+    def _read_smi(self):
+        for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
+                sm, smax, power = float(parts[1]), float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            for n, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+            reasons = {n for n, val in zip(self.REASON_NAMES, parts[5:9]) if val.lower() == "active"}
+            self.samples.append((time.perf_counter(), sm, smax, power, reasons))
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
+    def stop(self):
+        self._stop.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if self.source is None:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        t0 = self.t0 if self.t0 is not None else float("-inf")
+        t1 = self.t1 if self.t1 is not None else float("inf")
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:
+            return None
+        reasons = set()
+        for s in inside:
+            reasons |= s[4]
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": max(s[2] for s in inside),
+                "power_w_median": statistics.median(s[3] for s in inside), "samples": len(inside),
+                "reasons": sorted(reasons), "source": self.source,
+                "window_ms": (t1 - t0) * 1e3 if self.t0 is not None and self.t1 is not None else None}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -322,16 +409,17 @@ def gpu_arm(args, w):
     if fa.check_status() != 0:
         raise RuntimeError("device status word set during warm-up")
 
-    sampler = ClockSampler(local if ws > 1 else 0) if not args.no_clocks else None
+    sampler = ClockSampler(dev) if not args.no_clocks else None
     if sampler is not None:
         time.sleep(0.3)  # let the sampler start before the timed region
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    in_bytes = q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size()
-    small = in_bytes < L2_BYTES
+    small = l2_flush_needed(q, k, v)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    if sampler is not None:
+        sampler.mark_start()
     if not small:
         start.record(stream)
         for _ in range(args.steps):
@@ -352,6 +440,8 @@ def gpu_arm(args, w):
             end.synchronize()
             elapsed_ms += start.elapsed_time(end)
         del flush
+    if sampler is not None:
+        sampler.mark_end()
     if ws > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler is not None else None
@@ -479,8 +569,8 @@ def gpu_arm(args, w):
         cfg = {"workload": w.name, **{k: v for k, v in w.describe().items() if k != "workload"},
                "flop_convention": ("4 d per kept (query, key) pair" if (w.nq > 0 or w.n_sink > 0) else
                                    "4 B Hq N^2 d, /2 causal; 4 B Hq d (N W - W^2/2) with a window"),
-               "l2": ("L2 flushed before every step (inputs smaller than L2); steps timed one by one" if small
-                      else "inputs larger than L2 (no flush needed)"),
+               "l2": ("L2 flushed before every step (inputs, or K and V, smaller than L2); steps timed one by one"
+                      if small else "inputs and K + V larger than L2 (no flush needed)"),
                "parallelism": f"replicas x{ws} (independent batches)"}
         if args.splits > 0:
             cfg["split_kv"] = args.splits
@@ -580,18 +670,22 @@ def softmax_arm(args, sw):
     for _ in range(args.warmup):
         step(x)
     torch.cuda.synchronize(dev)
-    sampler = ClockSampler(local if ws > 1 else 0) if not args.no_clocks else None
+    sampler = ClockSampler(dev) if not args.no_clocks else None
     if sampler is not None:
         time.sleep(0.3)
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if sampler is not None:
+        sampler.mark_start()
     ev0.record(stream)
     for _ in range(args.steps):
         step(x)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
+    if sampler is not None:
+        sampler.mark_end()
     if ws > 1:
         dist.barrier()
     ms = ev0.elapsed_time(ev1)

@@ -40,3 +40,30 @@ def test_softmax_bytes():
 
 def test_job_throughput_is_the_whole_job_over_the_slowest_rank():
     assert bench.job_tflops(4, 1e12, 10, 1000.0) == 4 * 1e12 * 10 / 1.0 / 1e12
+
+
+def test_l2_flush_decision_looks_at_k_and_v():
+    """Inputs larger than L2 in total but with K + V inside it (grouped-query attention)
+    still get an L2 flush before every step; the headline workload does not need one."""
+    import torch
+
+    def meta(w):
+        mk = lambda h, n: torch.empty((w.B, h, n, w.d), dtype=torch.bfloat16, device="meta")  # noqa: E731
+        return mk(w.Hq, w.Nq), mk(w.Hkv, w.N), mk(w.Hkv, w.N)
+
+    assert not bench.l2_flush_needed(*meta(workloads.BY_NUMBER[3]))
+    assert bench.l2_flush_needed(*meta(workloads.BY_NUMBER[4]))   # K + V = 64 MiB
+    assert bench.l2_flush_needed(*meta(workloads.BY_NUMBER[2]))   # everything fits
+
+
+def test_clock_sampler_keeps_only_samples_inside_the_timed_region():
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.samples = [(0.5, 1000.0, 1965.0, 300.0, set()), (1.0, 1965.0, 1965.0, 700.0, {"sw_power_cap"}),
+                 (1.5, 1900.0, 1965.0, 800.0, set()), (3.0, 800.0, 1965.0, 200.0, {"hw_slowdown"})]
+    s.proc = s.thread = None
+    s.source = "test"
+    import threading
+    s._stop = threading.Event()
+    s.t0, s.t1 = 0.9, 2.0
+    c = s.stop()
+    assert c["samples"] == 2 and c["sm_mhz"] == (1965.0 + 1900.0) / 2 and c["reasons"] == ["sw_power_cap"]
