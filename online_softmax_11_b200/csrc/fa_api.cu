@@ -35,6 +35,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
   fa::OnceOnSuccess once;
   int num_sms = 0;
+  bool tc_ok = false;  // the tensor-core kernels were built with the launch register count they assume
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -45,39 +46,55 @@ int current_device(int* dev) {
   return FA_OK;
 }
 
+// Shared-memory size, and a check of the launch register count: the kernel re-splits its
+// registers between warpgroups with setmaxnreg, and the shares add up to exactly
+// kThreads x kLaunchRegs.  A build whose launch count differs would leave a register
+// request unsatisfiable, so such a kernel is refused here instead of launched.
+template <typename K>
+cudaError_t prepare_tc_kernel(K kernel, int smem_bytes, bool* regs_ok) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes a;
+  e = cudaFuncGetAttributes(&a, kernel);
+  if (e != cudaSuccess) return e;
+  if (a.numRegs > static_cast<int>(fa::tc::kLaunchRegs) || a.maxThreadsPerBlock < fa::tc::kThreads) *regs_ok = false;
+  return cudaSuccess;
+}
+
 template <int D, bool kSplit, bool kSinks>
-cudaError_t set_tc_smem() {
-  cudaError_t e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, fa::tc::Layout<D>::kSmemLaunch);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, fa::tc::Layout<D>::kSmemLaunch);
+cudaError_t set_tc_attributes(bool* regs_ok) {
+  constexpr int kSmem = fa::tc::Layout<D>::kSmemLaunch;
+  cudaError_t e = prepare_tc_kernel(fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, false>, kSmem, regs_ok);
+  if (e == cudaSuccess) e = prepare_tc_kernel(fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, true>, kSmem, regs_ok);
   return e;
 }
 
+struct TcMaps {
+  CUtensorMap q, k, v, o;
+};
+
 template <int D, bool kSplit, bool kSinks>
-void launch_tc_kernel(bool cap, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                      const fa::tc::Params& p, cudaStream_t s) {
+void launch_tc_kernel(bool cap, unsigned grid, const TcMaps& m, const fa::tc::Params& p, cudaStream_t s) {
   constexpr int kSmem = fa::tc::Layout<D>::kSmemLaunch;
   if (cap)
-    fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, true><<<grid, fa::tc::kThreads, kSmem, s>>>(mq, mk, mv, p);
+    fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, true><<<grid, fa::tc::kThreads, kSmem, s>>>(m.q, m.k, m.v, m.o, p);
   else
-    fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, false><<<grid, fa::tc::kThreads, kSmem, s>>>(mq, mk, mv, p);
+    fa::tc::fa_fwd_tc_kernel<D, kSplit, kSinks, false><<<grid, fa::tc::kThreads, kSmem, s>>>(m.q, m.k, m.v, m.o, p);
 }
 
 template <int D>
-void launch_tc_variant(bool split, bool sinks, bool cap, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mk,
-                       const CUtensorMap& mv, const fa::tc::Params& p, cudaStream_t s) {
+void launch_tc_variant(bool split, bool sinks, bool cap, unsigned grid, const TcMaps& m, const fa::tc::Params& p,
+                       cudaStream_t s) {
   if (split) {
-    if (sinks) launch_tc_kernel<D, true, true>(cap, grid, mq, mk, mv, p, s);
-    else launch_tc_kernel<D, true, false>(cap, grid, mq, mk, mv, p, s);
+    if (sinks) launch_tc_kernel<D, true, true>(cap, grid, m, p, s);
+    else launch_tc_kernel<D, true, false>(cap, grid, m, p, s);
   } else {
-    if (sinks) launch_tc_kernel<D, false, true>(cap, grid, mq, mk, mv, p, s);
-    else launch_tc_kernel<D, false, false>(cap, grid, mq, mk, mv, p, s);
+    if (sinks) launch_tc_kernel<D, false, true>(cap, grid, m, p, s);
+    else launch_tc_kernel<D, false, false>(cap, grid, m, p, s);
   }
 }
 
-int prepare_device(int dev, int* num_sms = nullptr) {
+int prepare_device(int dev, int* num_sms = nullptr, bool* tc_ok = nullptr) {
   DeviceState& st = g_dev[dev];
   const int status = st.once.run([&]() -> int {
     cudaDeviceProp prop;
@@ -90,14 +107,16 @@ int prepare_device(int dev, int* num_sms = nullptr) {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(fa::dec::fa_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                fa::dec::Smem<64>::kAlloc);
-    if (e == cudaSuccess) e = set_tc_smem<128, false, false>();
-    if (e == cudaSuccess) e = set_tc_smem<128, true, false>();
-    if (e == cudaSuccess) e = set_tc_smem<128, false, true>();
-    if (e == cudaSuccess) e = set_tc_smem<128, true, true>();
-    if (e == cudaSuccess) e = set_tc_smem<64, false, false>();
-    if (e == cudaSuccess) e = set_tc_smem<64, true, false>();
-    if (e == cudaSuccess) e = set_tc_smem<64, false, true>();
-    if (e == cudaSuccess) e = set_tc_smem<64, true, true>();
+    bool regs_ok = true;
+    if (e == cudaSuccess) e = set_tc_attributes<128, false, false>(&regs_ok);
+    if (e == cudaSuccess) e = set_tc_attributes<128, true, false>(&regs_ok);
+    if (e == cudaSuccess) e = set_tc_attributes<128, false, true>(&regs_ok);
+    if (e == cudaSuccess) e = set_tc_attributes<128, true, true>(&regs_ok);
+    if (e == cudaSuccess) e = set_tc_attributes<64, false, false>(&regs_ok);
+    if (e == cudaSuccess) e = set_tc_attributes<64, true, false>(&regs_ok);
+    if (e == cudaSuccess) e = set_tc_attributes<64, false, true>(&regs_ok);
+    if (e == cudaSuccess) e = set_tc_attributes<64, true, true>(&regs_ok);
+    st.tc_ok = regs_ok;
     if (e == cudaSuccess)  // two 1024-thread softmax blocks per SM: keep L1 small, shared memory is tiny
       e = cudaFuncSetAttribute(fa::smx::softmax_online_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 10);
     // the fp32 path needs up to 4 * (32 d + 32 (d + 1) + 32 d) bytes = 49280 at d = 128
@@ -115,6 +134,7 @@ int prepare_device(int dev, int* num_sms = nullptr) {
     return FA_OK;
   });
   if (num_sms) *num_sms = st.num_sms;
+  if (tc_ok) *tc_ok = st.tc_ok;
   return status;
 }
 
@@ -135,18 +155,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [heads, N, d] bf16 tensor viewed as 3-D (d, N, heads); boxes of 64 columns x 128 rows
-// with 128-byte swizzle, which is the canonical K-major (Q, K) and MN-major (V) operand
-// layout of tcgen05.mma.  Rows past N read as zero.
-int make_map(CUtensorMap* map, const void* base, int heads, int N, int d, unsigned box_rows = 128) {
+// [heads, N, d] bf16 tensor viewed as 3-D (d, N, heads) with boxes of 64 columns x
+// box_rows rows and 128-byte swizzle, which is the canonical K-major (Q, K) and MN-major
+// (V) operand layout of tcgen05.mma and the kernel's O staging layout.  Loads read rows
+// past N as zero; stores do not write them.
+int make_map(CUtensorMap* map, const void* base, int heads, int N, int d, unsigned box_rows = 128,
+             unsigned box_cols = 64, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(heads)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t box[3] = {box_cols, box_rows, 1};
   const cuuint32_t elem_strides[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem_strides,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
   return FA_OK;
@@ -282,20 +304,25 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
               float* o_part, float* lse_part, cudaStream_t s) {
   int rc;
   int dev, num_sms = 0;
+  bool tc_ok = false;
   if ((rc = current_device(&dev)) != FA_OK) return rc;
-  if ((rc = prepare_device(dev, &num_sms)) != FA_OK) return rc;
+  if ((rc = prepare_device(dev, &num_sms, &tc_ok)) != FA_OK) return rc;
   if (Nk == 0) return launch_no_keys(o, lse, static_cast<long long>(B) * Hq * Nq, d, s);
   if ((Hq / Hkv) * static_cast<long long>(Nq) <= fa::dec::kRows)
     return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, n_sink, softcap, num_splits,
                          o_part, lse_part, s);
 
-  CUtensorMap mq, mk, mv;
-  if ((rc = make_map(&mq, q, B * Hq, Nq, d)) != FA_OK) return rc;
-  if ((rc = make_map(&mk, k, B * Hkv, Nk, d)) != FA_OK) return rc;
-  if ((rc = make_map(&mv, v, B * Hkv, Nk, d)) != FA_OK) return rc;
-
+  if (!tc_ok) return FA_ERR_UNSUPPORTED;  // never launch a kernel whose register split cannot be met
   namespace tc = fa::tc;
   const bool split = num_splits >= 1;
+  TcMaps maps;
+  if ((rc = make_map(&maps.q, q, B * Hq, Nq, d, tc::BM)) != FA_OK) return rc;
+  if ((rc = make_map(&maps.k, k, B * Hkv, Nk, d, tc::BN)) != FA_OK) return rc;
+  if ((rc = make_map(&maps.v, v, B * Hkv, Nk, d, tc::BN)) != FA_OK) return rc;
+  if (split)
+    maps.o = maps.q;  // the split-KV epilogue writes fp32 partials without TMA
+  else if ((rc = make_map(&maps.o, o, B * Hq, Nq, d, tc::BM)) != FA_OK)
+    return rc;
   tc::Params p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -330,9 +357,9 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   const bool sinks = p.n_sink > 0;
   const bool cap = p.use_softcap != 0;
   if (d == 128)
-    launch_tc_variant<128>(split, sinks, cap, grid, mq, mk, mv, p, s);
+    launch_tc_variant<128>(split, sinks, cap, grid, maps, p, s);
   else
-    launch_tc_variant<64>(split, sinks, cap, grid, mq, mk, mv, p, s);
+    launch_tc_variant<64>(split, sinks, cap, grid, maps, p, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   if (split) {

@@ -9,11 +9,20 @@
 //                                              uses positions in the full sequence)
 //   m_new = max(m, rowmax s)                   one query row per thread: row max and sum
 //   P     = exp(s - m), l = alpha l + sum P    are thread-local; P rounded to bf16 and
-//                                              written back into TMEM over S_i
-//   O_i   = alpha O_i + P V_j                  tcgen05.mma, A = P from TMEM, B = V from
-//                                              shared memory (MN-major, no transpose)
+//                                              stored to shared memory
+//   O_i   = alpha O_i + P V_j                  tcgen05.mma, A = P and B = V (MN-major, no
+//                                              transpose) from shared memory
 // and finally O_i / l (bf16) and LSE = m + ln l (fp32), each written to HBM once.  The
 // score matrix never leaves the SM.
+//
+// Pipeline.  The softmax reads its whole 128-score row of S from TMEM with one load and
+// says so at once; S of the next key tile can then be computed into the same TMEM
+// columns while the softmax is still exponentiating, so per query tile the tensor core
+// runs S_{j+1} in the shadow of softmax_j and P_j V_j right after it (P lives in shared
+// memory, one 32 KB buffer per query tile, in two 64-key slabs with their own barriers so
+// each half's P.V starts as soon as that half is stored).  The two query tiles run the
+// same chain independently and share the tensor core and the K/V ring.  The ring streams
+// K one tile ahead of V (K_0, K_1, V_0, K_2, V_1, ...), the order the MMAs consume them.
 //
 // Persistent CTAs, one per SM.  The work tiles are grouped in units of two query-tile
 // pairs of one head, {q-pair n-1-p, q-pair p}; under a causal mask the two halves of a
@@ -22,17 +31,17 @@
 // CTAs running at the same time share the K/V of a few heads in L2.
 //
 // Roles (384 threads = 3 warpgroups):
-//   warpgroup 0  softmax for Q0 (thread t owns TMEM lane t = query row t), epilogue of Q0
-//   warpgroup 1  softmax for Q1, epilogue of Q1
-//   warpgroup 2  warp 8: TMA producer (Q0/Q1 per work tile, then K_j, V_j into a ring of
-//                shared-memory slots); warps 9 and 10: one MMA-issuing thread per query
+//   warpgroup 0  softmax for Q0 (thread t owns TMEM lane t = query row t), the lazy
+//                rescale of its row of O, and the epilogue of Q0
+//   warpgroup 1  the same for Q1
+//   warpgroup 2  warp 8: TMA producer (Q0/Q1 per work tile, then K and V tiles into a ring
+//                of shared-memory slots); warps 9 and 10: one MMA-issuing thread per query
 //                tile (warp 9 also owns the TMEM allocation); warp 11 idle.
 // With 12 warps, at most 3 share an SM sub-partition, so each thread gets up to 168
 // registers: enough for a softmax thread to hold its whole 128-score row.
-// The two query tiles ping-pong: while one warpgroup exponentiates S_0, the tensor core
-// computes P_1 V and S_1 for the other.  Across work tiles the pipeline does not drain:
-// the K/V ring keeps streaming, and a warpgroup's epilogue of tile w overlaps the other
-// warpgroup's last key tile and the first MMAs of tile w+1.
+// Epilogue: O / l is written as bf16 into the query tile's P buffer (free once the last
+// P.V has completed) in the 128-byte-swizzled layout of the O tensor map and stored with
+// TMA, one 64-column slab per store.
 //
 // Online-softmax details:
 //   * Scores are handled in log2 units, u = s * scale * log2(e), so P = exp2(u - m) is one
@@ -41,8 +50,8 @@
 //     grows by more than kRescaleLog2 (2^8); P then stays <= 256, and O and l always share
 //     the same (possibly stale) reference, so the result is still exact up to rounding
 //     (Module 16, 16.2: the max subtraction is about range, not correctness).  When it
-//     moves, the row of O in TMEM is multiplied by alpha = exp2(m_old - m_new) before the
-//     next P V product is issued.
+//     moves, the row of O in TMEM is multiplied by alpha = exp2(m_old - m_new) once the
+//     previous tile's P.V has landed and before this tile's P.V is released.
 //   * A row whose maximum is still -inf uses 0 as its reference, so masked scores give
 //     P = 0 and never NaN; alpha is 0 in that case (the guard of oxios'
 //     FlashAttention::attention for the first rescale).
@@ -71,6 +80,7 @@ constexpr int kTmemCols = 512;                // S0 | S1 | O0 | O1, 128 columns 
 constexpr float kRescaleLog2 = 8.0f;          // lazy-rescale threshold (log2 units)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr uint32_t kLaunchRegs = 168;  // 384 threads, one CTA per SM
 
 template <int D>
 struct Layout {
@@ -78,23 +88,30 @@ struct Layout {
   static constexpr int kHalves = D / 64;               // 64-column (128-byte) slabs per row
   static constexpr int kHalfBytes = 128 * 128;         // one slab of a 128-row tile
   static constexpr int kTileBytes = 128 * D * 2;       // a Q, K or V tile
-  static constexpr int kStages = D == 128 ? 4 : 8;     // K/V ring slots
+  static constexpr int kStages = D == 128 ? 3 : 8;     // K/V ring slots
+  static constexpr int kPBytes = 128 * BN * 2;         // P of one query tile (bf16, 128 x 128)
   static constexpr int kQOff = 0;
-  static constexpr int kRingOff = kQOff + NQ * kTileBytes;
+  static constexpr int kPOff = kQOff + NQ * kTileBytes;
+  static constexpr int kRingOff = kPOff + NQ * kPBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
   // barriers
   static constexpr int kBarQFull = 0;                     // [NQ]
   static constexpr int kBarQEmpty = kBarQFull + NQ;       // [NQ]
   static constexpr int kBarKvFull = kBarQEmpty + NQ;      // [kStages]
   static constexpr int kBarKvEmpty = kBarKvFull + kStages;
-  static constexpr int kBarSFull = kBarKvEmpty + kStages; // [NQ]
-  static constexpr int kBarPFull = kBarSFull + NQ;        // [NQ][2]: P of key half 0 / 1 stored
-  static constexpr int kBarOFull = kBarPFull + 2 * NQ;    // [NQ]
-  static constexpr int kBarDrain = kBarOFull + NQ;
+  static constexpr int kBarSFull = kBarKvEmpty + kStages; // [NQ]: S computed
+  static constexpr int kBarSFree = kBarSFull + NQ;        // [NQ]: S read into registers
+  static constexpr int kBarPFull = kBarSFree + NQ;        // [NQ][2]: P of key half 0 / 1 stored
+  static constexpr int kBarPFree = kBarPFull + 2 * NQ;    // [NQ][2]: ... and read by its P.V
+  static constexpr int kBarOFull = kBarPFree + 2 * NQ;    // [NQ]
+  static constexpr int kBarStgFull = kBarOFull + NQ;      // [NQ]: O staged in shared memory
+  static constexpr int kBarStgEmpty = kBarStgFull + NQ;   // [NQ]: ... and read by its TMA store
+  static constexpr int kBarDrain = kBarStgEmpty + NQ;
   static constexpr int kNumBars = kBarDrain + NQ;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // u32 tmem base, int abort flag
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;         // slack for 1024-byte alignment
+  static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
   // TMEM columns: S_i at 128 i, O_i at 256 + 128 i
   __device__ static constexpr uint32_t col_s(int i) { return static_cast<uint32_t>(i) * 128u; }
   __device__ static constexpr uint32_t col_o(int i) { return 256u + static_cast<uint32_t>(i) * 128u; }
@@ -201,23 +218,25 @@ enum class PMode {
 
 constexpr int kHalf = BN / 2;  // the softmax works on 64-score halves of a row
 
-// P = exp2(u - m) for 64 scores of this thread's row, written to TMEM as bf16 pairs
-// (32 keys = 16 columns per chunk) at taddr_p.  Returns the fp32 sum of these P.
+// P = exp2(u - m) for 64 scores of this thread's row (s[0 .. 63]), rounded to bf16 and
+// stored to this row of a 64-key slab of P in shared memory: 8 chunks of 8 keys (16 B),
+// chunk c at 16 (c ^ (row & 7)) -- the 128-byte swizzle the tensor core reads K-major
+// operands in.  Returns the fp32 sum of these P.
 template <PMode kMode>
-__device__ __forceinline__ float make_p(const float (&s)[kHalf], uint32_t taddr_p, float scale_log2, float cap_inner,
+__device__ __forceinline__ float make_p(const float* s, uint8_t* prow, int rsw, float scale_log2, float cap_inner,
                                         float cap_outer, float m_use) {
   const float2 negm = make_float2(-m_use, -m_use);
   float2 lsum0 = make_float2(0.f, 0.f), lsum1 = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int cb = 0; cb < kHalf / 32; ++cb) {
-    uint32_t packed[16];
+  for (int c = 0; c < kHalf / 8; ++c) {
+    uint32_t packed[4];
 #pragma unroll
-    for (int x = 0; x < 16; ++x) {
-      const float2 sv = make_float2(s[cb * 32 + 2 * x], s[cb * 32 + 2 * x + 1]);
+    for (int x = 0; x < 4; ++x) {
+      const float2 sv = make_float2(s[c * 8 + 2 * x], s[c * 8 + 2 * x + 1]);
       float2 e;
       if constexpr (kMode == PMode::kPlainMixed || kMode == PMode::kPlainMufu) {
         const float2 u = __ffma2_rn(sv, make_float2(scale_log2, scale_log2), negm);
-        if (kMode == PMode::kPlainMixed && (x & 3) == 3)  // one pair in four on the FMA pipe
+        if (kMode == PMode::kPlainMixed && x == 3)  // one pair in four on the FMA pipe
           e = exp2_fma_pair(u);
         else
           e = ex2_pair(u);
@@ -236,33 +255,33 @@ __device__ __forceinline__ float make_p(const float (&s)[kHalf], uint32_t taddr_
         lsum0 = __fadd2_rn(lsum0, e);
       packed[x] = pack_bf16x2(e.x, e.y);
     }
-    tmem_st16(taddr_p + cb * 16, packed);
+    *reinterpret_cast<uint4*>(prow + ((c ^ rsw) << 4)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
   }
   const float2 lsum = __fadd2_rn(lsum0, lsum1);
   return lsum.x + lsum.y;
 }
 
-// 64 scores of the row (tile columns c0 .. c0+63) from TMEM, masked when the tile needs a
-// mask: -inf above column c_hi and in the hole [h_lo, h_hi) of columns below the window
-// that are not attention sinks.  sink_cols (uniform over the tile) says whether the tile
-// holds sink columns at all; without them the hole starts at column 0.  kSinks = false
-// (no sinks in the launch) compiles only that second form.
+// The 128 scores of the row for one key tile from TMEM (one load, one wait), masked when
+// the tile needs a mask: -inf above column c_hi and in the hole [h_lo, h_hi) of columns
+// below the window that are not attention sinks.  sink_cols (uniform over the tile) says
+// whether the tile holds sink columns at all; without them the hole starts at column 0.
+// kSinks = false (no sinks in the launch) compiles only that second form.
 template <bool kSinks>
-__device__ __forceinline__ void load_half(uint32_t taddr, int c0, bool need_mask, bool sink_cols, int h_lo,
-                                          int h_hi, int c_hi, float (&s)[kHalf]) {
-  uint32_t r[kHalf];
-  tmem_ld64_wait(taddr, r);
+__device__ __forceinline__ void load_row(uint32_t taddr, bool need_mask, bool sink_cols, int h_lo, int h_hi,
+                                         int c_hi, float (&s)[BN]) {
+  uint32_t r[BN];
+  tmem_ld128_wait(taddr, r);
 #pragma unroll
-  for (int c = 0; c < kHalf; ++c) s[c] = __uint_as_float(r[c]);
+  for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
   if (need_mask) {
     if (kSinks && sink_cols) {
       const uint32_t hole = static_cast<uint32_t>(h_hi - h_lo);
 #pragma unroll
-      for (int c = 0; c < kHalf; ++c)
-        s[c] = (static_cast<uint32_t>(c0 + c - h_lo) < hole || c0 + c > c_hi) ? -CUDART_INF_F : s[c];
+      for (int c = 0; c < BN; ++c)
+        s[c] = (static_cast<uint32_t>(c - h_lo) < hole || c > c_hi) ? -CUDART_INF_F : s[c];
     } else {
 #pragma unroll
-      for (int c = 0; c < kHalf; ++c) s[c] = (c0 + c < h_hi || c0 + c > c_hi) ? -CUDART_INF_F : s[c];
+      for (int c = 0; c < BN; ++c) s[c] = (c < h_hi || c > c_hi) ? -CUDART_INF_F : s[c];
     }
   }
 }
@@ -419,7 +438,8 @@ __device__ __forceinline__ void for_each_tile(const Params& p, F&& f) {
 template <int D, bool kSplit, bool kSinks, bool kCap>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const Params p) {
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                     const Params p) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -437,9 +457,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[L::kBarQFull + i], 1);
       mbar_init(&bars[L::kBarQEmpty + i], 1);
       mbar_init(&bars[L::kBarSFull + i], 1);
-      mbar_init(&bars[L::kBarPFull + 2 * i], 128);
-      mbar_init(&bars[L::kBarPFull + 2 * i + 1], 128);
+      mbar_init(&bars[L::kBarSFree + i], BM);
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(&bars[L::kBarPFull + 2 * i + h], BM);
+        mbar_init(&bars[L::kBarPFree + 2 * i + h], 1);
+      }
       mbar_init(&bars[L::kBarOFull + i], 1);
+      mbar_init(&bars[L::kBarStgFull + i], BM);
+      mbar_init(&bars[L::kBarStgEmpty + i], 1);
     }
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&bars[L::kBarKvFull + s], 1);
@@ -481,20 +506,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                         w.bh);
           ++q_cnt[i];
         }
+        // ring order K_0, then (K_{n+1}, V_n) per position, V_{T-1} last: each key tile's
+        // S is issued one tile ahead of its neighbour's P.V
         const int T = w.ks.count();
-        for (int n = 0; n < T; ++n) {
+        for (int x = 0; x < 2 * T; ++x) {
+          const bool is_v = x > 0 && (x == 2 * T - 1 || (x & 1) == 0);
+          const int n = is_v ? (x == 2 * T - 1 ? T - 1 : (x - 2) / 2) : (x == 0 ? 0 : (x + 1) / 2);
           const int j = w.ks.at(n);
-          for (int which = 0; which < 2; ++which) {
-            const int s = issued % L::kStages;
-            const uint32_t fill = issued / L::kStages;
-            if (!mbar_wait(&bars[L::kBarKvEmpty + s], (fill & 1u) ^ 1u, ctl)) return false;
-            uint8_t* dst = smem + L::kRingOff + s * L::kTileBytes;
-            mbar_arrive_expect_tx(&bars[L::kBarKvFull + s], L::kTileBytes);
-            for (int h = 0; h < L::kHalves; ++h)
-              tma_load_3d(dst + h * L::kHalfBytes, which ? &tmV : &tmK, &bars[L::kBarKvFull + s], h * 64, j * BN,
-                          w.kvh);
-            ++issued;
-          }
+          const int s = issued % L::kStages;
+          const uint32_t fill = issued / L::kStages;
+          if (!mbar_wait(&bars[L::kBarKvEmpty + s], (fill & 1u) ^ 1u, ctl)) return false;
+          uint8_t* dst = smem + L::kRingOff + s * L::kTileBytes;
+          mbar_arrive_expect_tx(&bars[L::kBarKvFull + s], L::kTileBytes);
+          for (int h = 0; h < L::kHalves; ++h)
+            tma_load_3d(dst + h * L::kHalfBytes, is_v ? &tmV : &tmK, &bars[L::kBarKvFull + s], h * 64, j * BN,
+                        w.kvh);
+          ++issued;
         }
         return true;
       });
@@ -509,30 +536,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if ((warp == kMmaWarp || warp == kMmaWarp + 1) && lane == 0) {
       // =========================== MMA issuers ===========================
-      // One issuing thread per query tile (warp 9: Q0, warp 10: Q1).  Each thread's chain
-      // P_i V -> Q_i K^T is ordered by issue order (S_i overwrites the columns P_i was read
-      // from); the two chains are independent, so one thread's waits and commits overlap
-      // the other's MMAs.  Every K/V slot is released by both issuers (count 2): with a
-      // commit after the MMAs that read it, or a plain arrive when its query tile does not
-      // use that key tile (after the fill has landed, so a thread can never arrive ahead
-      // into the slot's next phase).
+      // One issuing thread per query tile (warp 9: Q0, warp 10: Q1).  P lives in shared
+      // memory, so S of the next key tile only has to wait until the softmax has read the
+      // current S into registers: per position n the thread issues S_n (once S_{n-1} is
+      // read), then P_{n-1} V_{n-1} in two 64-key halves (as each half of P is stored).
+      // Every K/V slot is released by both issuers (count 2): with a commit after the MMAs
+      // that read it, or a plain arrive when its query tile does not use that key tile
+      // (after the fill has landed, so a thread can never arrive ahead into the slot's
+      // next phase).
       const int i = warp - kMmaWarp;
-      constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);  // Q (K-major) x K (K-major)
-      constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, D, 0, 1);  // P (TMEM) x V (MN-major)
+      constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);   // Q (K-major) x K (K-major)
+      constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, D, 0, 1);   // P (K-major) x V (MN-major)
       // Descriptor of the first 16-column K step of each operand tile; later steps add
-      // their byte offset / 16 to the start-address field (no carry: addresses < 256 KB),
-      // inside mma_ss_kloop / mma_ts_kloop8.
+      // their byte offset / 16 to the start-address field (no carry: addresses < 256 KB).
       const uint64_t dq = smem_desc_sw128(smem_addr(smem + L::kQOff + i * L::kTileBytes), 16, 1024);
+      const uint64_t dpv = smem_desc_sw128(smem_addr(smem + L::kPOff + i * L::kPBytes), 16, 1024);
       const uint64_t dring = smem_desc_sw128(smem_addr(smem + L::kRingOff), 16, 1024);
       const uint64_t dvring = smem_desc_sw128(smem_addr(smem + L::kRingOff), L::kHalfBytes, 1024);
       const uint32_t d_s = tmem + L::col_s(i);
       const uint32_t d_o = tmem + L::col_o(i);
-      uint32_t q_cnt = 0, p_phase = 0;
+      uint32_t q_cnt = 0, g_s = 0, g_p = 0;
       int used = 0;  // ring loads consumed before the current work tile
 
       for_each_tile(p, [&](const WorkTile& w) {
         const TileRange& t = w.tr(i);
-        uint32_t o_acc = 0;
         const int T = w.ks.count();
         // this query tile's key tiles as positions in the work tile's sequence: each of
         // its runs lies inside one run of the sequence, so it is a run of positions too
@@ -553,59 +580,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int n_first = sa1 > sa0 ? sa0 : sb0;
         const int n_last = sb1 > sb0 ? sb1 - 1 : sa1 - 1;
-        for (int n = 0; n <= T; ++n) {
-          // position n: S of the n-th key tile; position n - 1: its P.V
-          const bool use_s = n < T && ((kSinks && n >= sa0 && n < sa1) || (n >= sb0 && n < sb1));
-          const bool use_pv = n > 0 && ((kSinks && n - 1 >= sa0 && n - 1 < sa1) || (n - 1 >= sb0 && n - 1 < sb1));
-          const int kidx = used + 2 * n;
-          const int vidx = kidx - 1;
-          const int kslot = kidx % L::kStages;
+        auto uses = [&](int n) { return (kSinks && n >= sa0 && n < sa1) || (n >= sb0 && n < sb1); };
+        uint32_t o_acc = 0;
+        // V_n: O_i (+)= P_i V_n in two halves of 64 keys, or release
+        auto pv = [&](int n) -> bool {
+          const int vidx = used + (n == T - 1 ? 2 * T - 1 : 2 * n + 2);
           const int vslot = vidx % L::kStages;
-          // TMA -> MMA hand-offs (K, V, Q) need only the mbarrier (both sides are async
-          // proxy on shared memory).  P, written to tensor memory by the softmax warps'
-          // tcgen05.st, also needs tcgen05.fence::after_thread_sync after its barrier.
-          if (n > 0) {
-            if (use_pv) {
-              if (!mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
-              // O_i (+)= P_i V in two halves of 64 keys, each as soon as the softmax has
-              // stored that half of P (the second half of the softmax overlaps the first
-              // half's MMAs): A = 16 keys of P = 8 TMEM columns per step; B = 16 key rows
-              // of V (128 B each); the two 64-column slabs of V are kHalfBytes apart
-              const uint64_t dv = dvring + ((vslot * L::kTileBytes) >> 4);
-              if (!mbar_wait(&bars[L::kBarPFull + 2 * i], p_phase, ctl)) return false;
-              tc_fence_after();
-              mma_ts_kloop4(d_o, d_s, dv, kIdescPV, o_acc);
-              if (!mbar_wait(&bars[L::kBarPFull + 2 * i + 1], p_phase, ctl)) return false;
-              p_phase ^= 1u;
-              tc_fence_after();
-              mma_ts_kloop4(d_o, d_s + 32, dv + 512, kIdescPV, 1u);
-              o_acc = 1;
-              if (n - 1 == n_last) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
-              mma_commit(&bars[L::kBarKvEmpty + vslot]);
-            } else {
-              // not used by this query tile: release it, but only once this fill has
-              // landed, so the arrive cannot be counted towards the slot's next fill
-              if (!mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
-              mbar_arrive(&bars[L::kBarKvEmpty + vslot]);
-            }
+          if (!mbar_wait(&bars[L::kBarKvFull + vslot], (vidx / L::kStages) & 1u, ctl)) return false;
+          if (!uses(n)) {
+            mbar_arrive(&bars[L::kBarKvEmpty + vslot]);
+            return true;
           }
-          if (n < T) {
-            if (use_s) {
-              if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
-              if (n == n_first) {  // first use of this work tile's Q_i
-                if (!mbar_wait(&bars[L::kBarQFull + i], q_cnt & 1u, ctl)) return false;
-                ++q_cnt;
-              }
-              mma_ss_kloop<D / 16>(d_s, dq, dring + ((kslot * L::kTileBytes) >> 4), kIdescS);
-              mma_commit(&bars[L::kBarSFull + i]);
-              if (n == n_last) mma_commit(&bars[L::kBarQEmpty + i]);  // Q_i no longer read
-              mma_commit(&bars[L::kBarKvEmpty + kslot]);
-            } else {
-              if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
-              mbar_arrive(&bars[L::kBarKvEmpty + kslot]);
-            }
+          const uint64_t dv = dvring + ((vslot * L::kTileBytes) >> 4);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            // P half h stored (by the softmax warps' generic-proxy stores, fenced for the
+            // async proxy) and, for half 0, O rescaled in TMEM
+            if (!mbar_wait(&bars[L::kBarPFull + 2 * i + h], g_p & 1u, ctl)) return false;
+            tc_fence_after();
+            // A = 16 keys of P (32 B of each 128-byte swizzled row; the halves are one
+            // 16 KB slab each); B = 16 key rows of V (128 B each; half 1 starts 64 rows in)
+            mma_ss_pv4(d_o, dpv + h * (L::kHalfBytes >> 4), dv + h * 512, kIdescPV, (o_acc | h) != 0u);
+            mma_commit(&bars[L::kBarPFree + 2 * i + h]);
           }
+          o_acc = 1;
+          if (n == n_last) mma_commit(&bars[L::kBarOFull + i]);  // O_i is final
+          mma_commit(&bars[L::kBarKvEmpty + vslot]);
+          ++g_p;
+          return true;
+        };
+        for (int n = 0; n < T; ++n) {
+          const int kidx = used + (n == 0 ? 0 : 2 * n - 1);
+          const int kslot = kidx % L::kStages;
+          if (!mbar_wait(&bars[L::kBarKvFull + kslot], (kidx / L::kStages) & 1u, ctl)) return false;
+          if (uses(n)) {
+            if (n == n_first) {  // first use of this work tile's Q_i
+              if (!mbar_wait(&bars[L::kBarQFull + i], q_cnt & 1u, ctl)) return false;
+              ++q_cnt;
+            }
+            if (g_s > 0) {  // the softmax has the previous S of this query tile in registers
+              if (!mbar_wait(&bars[L::kBarSFree + i], (g_s - 1) & 1u, ctl)) return false;
+              tc_fence_after();
+            }
+            mma_ss_kloop<D / 16>(d_s, dq, dring + ((kslot * L::kTileBytes) >> 4), kIdescS);
+            mma_commit(&bars[L::kBarSFull + i]);
+            if (n == n_last) mma_commit(&bars[L::kBarQEmpty + i]);  // Q_i no longer read
+            mma_commit(&bars[L::kBarKvEmpty + kslot]);
+            ++g_s;
+          } else {
+            mbar_arrive(&bars[L::kBarKvEmpty + kslot]);
+          }
+          if (n > 0 && !pv(n - 1)) return false;
         }
+        if (T > 0 && !pv(T - 1)) return false;
         used += 2 * T;
         return true;
       });
@@ -622,7 +649,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t colS = L::col_s(i);
     const uint32_t colO = L::col_o(i);
-    uint32_t s_phase = 0, o_phase = 0;
+    uint8_t* prow = smem + L::kPOff + i * L::kPBytes + trow * 128;  // this row of P (slab 0)
+    const int rsw = trow & 7;
+    uint32_t s_phase = 0, o_phase = 0, g = 0, stg_cnt = 0;
 
     for_each_tile(p, [&](const WorkTile& w) {
       const TileRange& t = w.tr(i);
@@ -656,30 +685,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h_lo = min(max(0, p.n_sink - k0), w_lo);
         const int h_hi = w_lo;
 
-        // Pass 1: row maximum (and minimum, for the soft-cap range check) over the two
-        // 64-score halves with three-input max: three chains over the columns whose exp2
-        // runs on the MUFU in unmasked plain tiles, one over those on the FMA pipe (pair 3
-        // of every 4, i.e. columns 8k+6, 8k+7), so the tile maximum's P can be recomputed
-        // with the very arithmetic that produced it.
+        // The whole row of S in registers with one TMEM load, then the row maximum (and
+        // minimum, for the soft-cap range check) with three-input max: three chains over
+        // the columns whose exp2 runs on the MUFU in unmasked plain tiles, one over those
+        // on the FMA pipe (pair 3 of every 4, i.e. columns 8k+6, 8k+7), so the tile
+        // maximum's P can be recomputed with the very arithmetic that produced it.
+        float s[BN];
+        load_row<kSinks>(lane_base + colS, need_mask, sink_cols, h_lo, h_hi, c_hi, s);
+        // S is in registers: the next key tile's S may overwrite it
+        tc_fence_before();
+        mbar_arrive(&bars[L::kBarSFree + i]);
         float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F, mx2 = -CUDART_INF_F, mx_emu = -CUDART_INF_F;
         float mn0 = CUDART_INF_F, mn1 = CUDART_INF_F;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float s[kHalf];
-          load_half<kSinks>(lane_base + colS + h * kHalf, h * kHalf, need_mask, sink_cols, h_lo, h_hi, c_hi, s);
+        for (int c = 0; c < BN; c += 8) {
+          mx0 = fmax3(mx0, s[c], s[c + 1]);
+          mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+          mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+          mx_emu = fmax3(mx_emu, s[c + 6], s[c + 7]);
+        }
+        if constexpr (kCap) {
 #pragma unroll
-          for (int c = 0; c < kHalf; c += 8) {
-            mx0 = fmax3(mx0, s[c], s[c + 1]);
-            mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
-            mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
-            mx_emu = fmax3(mx_emu, s[c + 6], s[c + 7]);
-          }
-          if constexpr (kCap) {
-#pragma unroll
-            for (int c = 0; c < kHalf; c += 4) {
-              mn0 = fmin3(mn0, s[c], s[c + 1]);
-              mn1 = fmin3(mn1, s[c + 2], s[c + 3]);
-            }
+          for (int c = 0; c < BN; c += 4) {
+            mn0 = fmin3(mn0, s[c], s[c + 1]);
+            mn1 = fmin3(mn1, s[c + 2], s[c + 3]);
           }
         }
         const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx_emu));
@@ -691,33 +720,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_tile = mx * p.scale_log2;
         const float m_new = fmaxf(m, m_tile);
 
+        // alpha: the factor O is rescaled by (when the warp has a row that moved its
+        // reference); applied below, after the first half of P, when half of the scores
+        // no longer occupy registers, and after the previous tile's P.V has landed.
+        float alpha = 1.0f;
+        bool rescale = false;
         if (!o_valid) {
           m = m_new;  // nothing accumulated yet: adopt the maximum as is
         } else {
           const bool need = m_new > m + kRescaleLog2;
-          if (__any_sync(0xffffffffu, need)) {
-            const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
-            if (need) {
-              l *= alpha;
-              lr *= alpha;
-              m = m_new;
-            }
-            uint32_t r[32];
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              tmem_ld32_wait(lane_base + colO + c * 32, r);
-#pragma unroll
-              for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-              tmem_st32(lane_base + colO + c * 32, r);
-            }
+          rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            alpha = ex2_approx(m - m_new);
+            l *= alpha;
+            lr *= alpha;
+            m = m_new;
           }
         }
         const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
 
-        // Pass 2: per half, reload the scores, P = exp2(u - m) into TMEM over columns
-        // [32 h, 32 h + 32) of S (already consumed: half 0 was reloaded first).
-        // lt: fp32 sum of this tile's P; pmax: the P of the tile maximum, recomputed with
-        // the same instructions as in make_p (so it is bit-identical to the value packed).
+        // P = exp2(u - m) per 64-key half into its shared-memory slab, once the previous
+        // tile's P.V half has read the slab.  lt: fp32 sum of this tile's P; pmax: the P of
+        // the tile maximum, recomputed with the same instructions as in make_p (so it is
+        // bit-identical to the value packed).
         float lt = 0.f, pmax;
         int wtier = 0;
         if constexpr (kCap) {
@@ -727,26 +752,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          float s[kHalf];
-          load_half<kSinks>(lane_base + colS + h * kHalf, h * kHalf, need_mask, sink_cols, h_lo, h_hi, c_hi, s);
-          const uint32_t tp = lane_base + colS + h * (kHalf / 2);
+          const float* sh = s + h * kHalf;
+          uint8_t* ph = prow + h * L::kHalfBytes;
+          // the previous tile's P.V half h has read this slab (the first wait of a fresh
+          // barrier passes: there is no previous tile)
+          if (!mbar_wait(&bars[L::kBarPFree + 2 * i + h], (g & 1u) ^ 1u, ctl)) return false;
           if constexpr (!kCap) {
             if (need_mask)
-              lt += make_p<PMode::kPlainMufu>(s, tp, p.scale_log2, 0.f, 0.f, m_use);
+              lt += make_p<PMode::kPlainMufu>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
             else
-              lt += make_p<PMode::kPlainMixed>(s, tp, p.scale_log2, 0.f, 0.f, m_use);
+              lt += make_p<PMode::kPlainMixed>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
           } else if (wtier == 0) {
-            lt += make_p<PMode::kCapShort>(s, tp, 0.f, p.cap_inner, p.cap_outer, m_use);
+            lt += make_p<PMode::kCapShort>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
           } else if (wtier == 1) {
-            lt += make_p<PMode::kCapLong>(s, tp, 0.f, p.cap_inner, p.cap_outer, m_use);
+            lt += make_p<PMode::kCapLong>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
           } else {
-            lt += make_p<PMode::kCapGeneral>(s, tp, 0.f, p.cap_inner, p.cap_outer, m_use);
+            lt += make_p<PMode::kCapGeneral>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
           }
-          // this half of P is in tensor memory: its P.V can start
-          tmem_wait_st();
+          fence_proxy_async_smem();  // the tensor core reads P through the async proxy
+          if (h == 0 && rescale) {
+            // O must hold the previous tile's whole P.V: its second half has landed once
+            // the slab of P half 1 is free (same barrier the second half waits on below)
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarPFree + 2 * i + 1], (g & 1u) ^ 1u, ctl)))
+              return false;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld32_wait(lane_base + colO + c * 32, r);
+#pragma unroll
+              for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+              tmem_st32(lane_base + colO + c * 32, r);
+            }
+            tmem_wait_st();
+          }
+          // this half of P is stored (and O rescaled): its P.V can start
           tc_fence_before();
           mbar_arrive(&bars[L::kBarPFull + 2 * i + h]);
         }
+        ++g;
         if constexpr (!kCap) {
           const float u = fmaf(mx, p.scale_log2, -m_use);
           pmax = (!need_mask && mx_emu == mx) ? exp2_fma_pair(make_float2(u, u)).x : ex2_approx(u);
@@ -800,7 +844,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row < p.Nq) p.lse_part[prow] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
         return true;
       }
-      __nv_bfloat16* orow = p.o + (static_cast<int64_t>(w.bh) * p.Nq + row) * D;
+      // O / lr as bf16 into this query tile's P buffer (free: the last P.V, which read
+      // it, has completed) in the 128-byte-swizzled layout of the O tensor map, then one
+      // thread stores it with TMA, one 64-column slab per store; rows past Nq fall
+      // outside the tensor and are not written.  The buffer is P again once the stores
+      // have read it.
+      uint8_t* stg = smem + L::kPOff + i * L::kPBytes + trow * 128;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
@@ -810,21 +859,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int x = 0; x < 32; ++x) r[x] = 0u;
         }
-        if (row < p.Nq) {
-          uint4 v4[4];
-          uint32_t* wp = reinterpret_cast<uint32_t*>(v4);
+        uint8_t* slab = stg + (c >> 1) * L::kHalfBytes;
 #pragma unroll
-          for (int x = 0; x < 16; ++x)
-            wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * inv, __uint_as_float(r[2 * x + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) dst[x] = v4[x];
+        for (int x = 0; x < 4; ++x) {
+          const int q = (c & 1) * 4 + x;  // 16-byte chunk of the 128-byte slab row
+          *reinterpret_cast<uint4*>(slab + ((q ^ rsw) << 4)) =
+              make_uint4(pack_bf16x2(__uint_as_float(r[8 * x]) * inv, __uint_as_float(r[8 * x + 1]) * inv),
+                         pack_bf16x2(__uint_as_float(r[8 * x + 2]) * inv, __uint_as_float(r[8 * x + 3]) * inv),
+                         pack_bf16x2(__uint_as_float(r[8 * x + 4]) * inv, __uint_as_float(r[8 * x + 5]) * inv),
+                         pack_bf16x2(__uint_as_float(r[8 * x + 6]) * inv, __uint_as_float(r[8 * x + 7]) * inv));
         }
       }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[L::kBarStgFull + i]);
       if (p.lse != nullptr && row < p.Nq)
         p.lse[static_cast<int64_t>(w.bh) * p.Nq + row] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+      bool ok = true;
+      if (trow == 0) {
+        ok = mbar_wait(&bars[L::kBarStgFull + i], stg_cnt & 1u, ctl);
+        if (ok) {
+          uint8_t* base = smem + L::kPOff + i * L::kPBytes;
+          for (int h = 0; h < L::kHalves; ++h) tma_store_3d(&tmO, base + h * L::kHalfBytes, h * 64, t.r0, w.bh);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(&bars[L::kBarStgEmpty + i]);
+        }
+      }
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, ok && mbar_wait(&bars[L::kBarStgEmpty + i], stg_cnt & 1u, ctl))) return false;
+      ++stg_cnt;
       return true;
     });
+    if (trow == 0) bulk_wait_group0();  // the last O stores have completed
   }
 
   // ---- teardown
