@@ -170,9 +170,11 @@ __device__ __forceinline__ float tanh_cap(float x) {
 // field.  The cubic's coefficients were fitted for minimum relative error on
 // [-1/2, 1/2] (Lawson's iteratively reweighted least squares): max relative error
 // 7.5e-5, below the 2^-9 of the bf16 rounding that P goes through next.  x is clamped at
-// -125 so the exponent cannot underflow; callers use this only on tiles with no masked
-// key (x > -inf), where 2^-125 is far below anything that can matter.
+// -125 so the exponent cannot underflow, and anything below -125 (a masked key's -inf
+// included) gives exactly 0, as the exponential unit does for -inf; between 2^-125 and
+// the unit's own underflow the two differ by less than anything that can matter.
 __device__ __forceinline__ float2 exp2_fma_pair(float2 x) {
+  const bool zx = x.x < -125.0f, zy = x.y < -125.0f;
   x.x = fmaxf(x.x, -125.0f);
   x.y = fmaxf(x.y, -125.0f);
   const float2 shifter = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
@@ -182,8 +184,8 @@ __device__ __forceinline__ float2 exp2_fma_pair(float2 x) {
   float2 q = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.2426111400f, 0.2426111400f));
   q = __ffma2_rn(q, f, make_float2(0.6932609677f, 0.6932609677f));
   q = __ffma2_rn(q, f, make_float2(0.9999280572f, 0.9999280572f));
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(r.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(r.y) << 23)));
+  return make_float2(zx ? 0.f : __uint_as_float(__float_as_uint(q.x) + (__float_as_uint(r.x) << 23)),
+                     zy ? 0.f : __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(r.y) << 23)));
 }
 
 __device__ __forceinline__ float2 ex2_pair(float2 x) { return make_float2(ex2_approx(x.x), ex2_approx(x.y)); }
@@ -209,8 +211,9 @@ __device__ __forceinline__ float2 tanh_small_pair(float2 x) {
 
 // How P is produced from the scores of one tile (chosen per tile, warp-uniformly).
 enum class PMode {
-  kPlainMixed,   // no soft-cap, no masked key: 3 of 4 pairs on ex2, 1 of 4 on the FMA pipe
-  kPlainMufu,    // no soft-cap, masked keys present (-inf -> exactly 0): all pairs on ex2
+  kPlainMixed,   // no soft-cap: 3 of 4 pairs on ex2, 1 of 4 on the FMA pipe (masked keys,
+                 // -inf, give exactly 0 on both); one code path for masked and unmasked
+                 // tiles keeps the loop small
   kCapShort,     // soft-cap, every |s * scale / cap| < 0.12
   kCapLong,      // soft-cap, every |s * scale / cap| < 0.3
   kCapGeneral,   // soft-cap, anything else (including masked keys)
@@ -234,7 +237,7 @@ __device__ __forceinline__ float make_p(const float* s, uint8_t* prow, int rsw, 
     for (int x = 0; x < 4; ++x) {
       const float2 sv = make_float2(s[c * 8 + 2 * x], s[c * 8 + 2 * x + 1]);
       float2 e;
-      if constexpr (kMode == PMode::kPlainMixed || kMode == PMode::kPlainMufu) {
+      if constexpr (kMode == PMode::kPlainMixed) {
         const float2 u = __ffma2_rn(sv, make_float2(scale_log2, scale_log2), negm);
         if (kMode == PMode::kPlainMixed && x == 3)  // one pair in four on the FMA pipe
           e = exp2_fma_pair(u);
@@ -687,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // The whole row of S in registers with one TMEM load, then the row maximum (and
         // minimum, for the soft-cap range check) with three-input max: three chains over
-        // the columns whose exp2 runs on the MUFU in unmasked plain tiles, one over those
+        // the columns whose exp2 runs on the MUFU in plain (no soft-cap) tiles, one over those
         // on the FMA pipe (pair 3 of every 4, i.e. columns 8k+6, 8k+7), so the tile
         // maximum's P can be recomputed with the very arithmetic that produced it.
         float s[BN];
@@ -758,10 +761,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // barrier passes: there is no previous tile)
           if (!mbar_wait(&bars[L::kBarPFree + 2 * i + h], (g & 1u) ^ 1u, ctl)) return false;
           if constexpr (!kCap) {
-            if (need_mask)
-              lt += make_p<PMode::kPlainMufu>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
-            else
-              lt += make_p<PMode::kPlainMixed>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
+            lt += make_p<PMode::kPlainMixed>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
           } else if (wtier == 0) {
             lt += make_p<PMode::kCapShort>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
           } else if (wtier == 1) {
@@ -793,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++g;
         if constexpr (!kCap) {
           const float u = fmaf(mx, p.scale_log2, -m_use);
-          pmax = (!need_mask && mx_emu == mx) ? exp2_fma_pair(make_float2(u, u)).x : ex2_approx(u);
+          pmax = (mx_emu == mx) ? exp2_fma_pair(make_float2(u, u)).x : ex2_approx(u);
         } else {
           const float xm = mx * p.cap_inner;
           if (wtier == 0)
