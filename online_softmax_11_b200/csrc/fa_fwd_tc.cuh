@@ -849,26 +849,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       // thread stores it with TMA, one 64-column slab per store; rows past Nq fall
       // outside the tensor and are not written.  The buffer is P again once the stores
       // have read it.
+      uint32_t r[D];
+      if (t.part) {
+        if constexpr (D == 128)
+          tmem_ld128_wait(lane_base + colO, r);
+        else
+          tmem_ld64_wait(lane_base + colO, r);
+      } else {  // no key at all for this query tile (fewer keys than queries, causal)
+#pragma unroll
+        for (int x = 0; x < D; ++x) r[x] = 0u;
+      }
       uint8_t* stg = smem + L::kPOff + i * L::kPBytes + trow * 128;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        if (t.part) {
-          tmem_ld32_wait(lane_base + colO + c * 32, r);
-        } else {  // no key at all for this query tile (fewer keys than queries, causal)
-#pragma unroll
-          for (int x = 0; x < 32; ++x) r[x] = 0u;
-        }
-        uint8_t* slab = stg + (c >> 1) * L::kHalfBytes;
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int q = (c & 1) * 4 + x;  // 16-byte chunk of the 128-byte slab row
-          *reinterpret_cast<uint4*>(slab + ((q ^ rsw) << 4)) =
-              make_uint4(pack_bf16x2(__uint_as_float(r[8 * x]) * inv, __uint_as_float(r[8 * x + 1]) * inv),
-                         pack_bf16x2(__uint_as_float(r[8 * x + 2]) * inv, __uint_as_float(r[8 * x + 3]) * inv),
-                         pack_bf16x2(__uint_as_float(r[8 * x + 4]) * inv, __uint_as_float(r[8 * x + 5]) * inv),
-                         pack_bf16x2(__uint_as_float(r[8 * x + 6]) * inv, __uint_as_float(r[8 * x + 7]) * inv));
-        }
+      for (int q = 0; q < D / 8; ++q) {  // 16-byte chunk q of the row: slab q / 8, chunk q % 8
+        const uint32_t* rq = r + 8 * q;
+        *reinterpret_cast<uint4*>(stg + (q >> 3) * L::kHalfBytes + (((q & 7) ^ rsw) << 4)) =
+            make_uint4(pack_bf16x2(__uint_as_float(rq[0]) * inv, __uint_as_float(rq[1]) * inv),
+                       pack_bf16x2(__uint_as_float(rq[2]) * inv, __uint_as_float(rq[3]) * inv),
+                       pack_bf16x2(__uint_as_float(rq[4]) * inv, __uint_as_float(rq[5]) * inv),
+                       pack_bf16x2(__uint_as_float(rq[6]) * inv, __uint_as_float(rq[7]) * inv));
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[L::kBarStgFull + i]);
