@@ -126,7 +126,8 @@ class ClockSampler:
     """SM clock, power and clock-event reasons sampled while the timed region runs.
 
     A background thread reads NVML every ``period_ms`` (read-only queries: current and
-    maximum SM clock, power draw, active clock-event reasons); ``nvidia-smi -lms`` is the
+    maximum SM clock, power draw, active clock-event reasons, and once the enforced power
+    limit); ``nvidia-smi -lms`` is the
     fallback when the NVML binding is missing.  Only samples taken between
     ``mark_start()`` and ``mark_end()`` (host times around the timed region, which ends
     with a device synchronisation) are reported.  The GPU is found by the UUID of the
@@ -145,6 +146,7 @@ class ClockSampler:
         self.proc = None
         self.thread = None
         self.source = None
+        self.power_limit_w = None  # enforced board power limit (read once, NVML only)
         self._stop = threading.Event()
         handle = self._nvml_handle(device)
         if handle is not None:
@@ -190,6 +192,10 @@ class ClockSampler:
                 "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
                 "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
         smax = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
+        try:
+            self.power_limit_w = pynvml.nvmlDeviceGetEnforcedPowerLimit(handle) / 1e3
+        except pynvml.NVMLError:
+            pass
         while not self._stop.is_set():
             t = time.perf_counter()
             try:
@@ -240,7 +246,9 @@ class ClockSampler:
         for s in inside:
             reasons |= s[4]
         return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": max(s[2] for s in inside),
-                "power_w_median": statistics.median(s[3] for s in inside), "samples": len(inside),
+                "sm_mhz_range": [min(s[1] for s in inside), max(s[1] for s in inside)],
+                "power_w_median": statistics.median(s[3] for s in inside), "power_limit_w": self.power_limit_w,
+                "samples": len(inside),
                 "reasons": sorted(reasons), "source": self.source,
                 "window_ms": (t1 - t0) * 1e3 if self.t0 is not None and self.t1 is not None else None}
 

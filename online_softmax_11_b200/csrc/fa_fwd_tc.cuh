@@ -264,7 +264,7 @@ __device__ __forceinline__ float make_p(const float* s, uint8_t* prow, int rsw, 
   return lsum.x + lsum.y;
 }
 
-// The 128 scores of the row for one key tile from TMEM (one load, one wait), masked when
+// The 128 scores of the row for one key tile from TMEM (two loads, one wait), masked when
 // the tile needs a mask: -inf above column c_hi and in the hole [h_lo, h_hi) of columns
 // below the window that are not attention sinks.  sink_cols (uniform over the tile) says
 // whether the tile holds sink columns at all; without them the hole starts at column 0.
@@ -273,7 +273,7 @@ template <bool kSinks>
 __device__ __forceinline__ void load_row(uint32_t taddr, bool need_mask, bool sink_cols, int h_lo, int h_hi,
                                          int c_hi, float (&s)[BN]) {
   uint32_t r[BN];
-  tmem_ld128_wait(taddr, r);
+  tmem_ld64x2_wait(taddr, r);
 #pragma unroll
   for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
   if (need_mask) {
@@ -688,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h_lo = min(max(0, p.n_sink - k0), w_lo);
         const int h_hi = w_lo;
 
-        // The whole row of S in registers with one TMEM load, then the row maximum (and
+        // The whole row of S in registers with one TMEM round trip, then the row maximum (and
         // minimum, for the soft-cap range check) with three-input max: three chains over
         // the columns whose exp2 runs on the MUFU in plain (no soft-cap) tiles, one over those
         // on the FMA pipe (pair 3 of every 4, i.e. columns 8k+6, 8k+7), so the tile

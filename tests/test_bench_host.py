@@ -62,8 +62,10 @@ def test_clock_sampler_keeps_only_samples_inside_the_timed_region():
                  (1.5, 1900.0, 1965.0, 800.0, set()), (3.0, 800.0, 1965.0, 200.0, {"hw_slowdown"})]
     s.proc = s.thread = None
     s.source = "test"
+    s.power_limit_w = 1000.0
     import threading
     s._stop = threading.Event()
     s.t0, s.t1 = 0.9, 2.0
     c = s.stop()
     assert c["samples"] == 2 and c["sm_mhz"] == (1965.0 + 1900.0) / 2 and c["reasons"] == ["sw_power_cap"]
+    assert c["sm_mhz_range"] == [1900.0, 1965.0] and c["power_limit_w"] == 1000.0
