@@ -757,9 +757,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < 2; ++h) {
           const float* sh = s + h * kHalf;
           uint8_t* ph = prow + h * L::kHalfBytes;
-          // the previous tile's P.V half h has read this slab (the first wait of a fresh
-          // barrier passes: there is no previous tile)
-          if (!mbar_wait(&bars[L::kBarPFree + 2 * i + h], (g & 1u) ^ 1u, ctl)) return false;
+          // the previous tile's P.V has read both slabs: one wait, on the second half's
+          // release, covers both, since the MMAs of one thread complete in the order they
+          // were issued (the first wait of a fresh barrier passes: there is no previous
+          // tile).  It has nearly always come by now, and every mbarrier test costs a
+          // shared-memory round trip, so the first half's release is not waited for.
+          if (h == 0 && !__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarPFree + 2 * i + 1], (g & 1u) ^ 1u, ctl)))
+            return false;
           if constexpr (!kCap) {
             lt += make_p<PMode::kPlainMixed>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
           } else if (wtier == 0) {
@@ -771,10 +775,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();  // the tensor core reads P through the async proxy
           if (h == 0 && rescale) {
-            // O must hold the previous tile's whole P.V: its second half has landed once
-            // the slab of P half 1 is free (same barrier the second half waits on below)
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarPFree + 2 * i + 1], (g & 1u) ^ 1u, ctl)))
-              return false;
+            // O must hold the previous tile's whole P.V: its second half has landed, as the
+            // wait above has shown
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {

@@ -98,7 +98,10 @@ __device__ __forceinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, cons
 }
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl ctl) {
   const uint32_t a = smem_addr(bar);
-  if (mbar_try_wait(a, parity)) return true;  // common case: no call, no timer read
+  // Most waits find the phase complete: a non-blocking test first is measurably cheaper
+  // there than the suspend-hinted form.
+  if (mbar_ready(bar, parity)) return true;
+  if (mbar_try_wait(a, parity)) return true;  // no call, no timer read
   return mbar_wait_slow(a, parity, ctl);
 }
 
