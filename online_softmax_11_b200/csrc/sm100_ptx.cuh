@@ -82,8 +82,8 @@ struct WaitCtl {
 // Wait for the phase with parity `parity` of `bar` to complete.  Returns false (after
 // recording FA_ERR_TIMEOUT in g_status and raising the CTA's abort flag) when the wait
 // takes longer than ctl.limit_ns, or when another thread of the CTA has aborted.
-// Inlined: a called function has one register allocation, which cannot fit kernels
-// whose warpgroups run with different register counts (setmaxnreg).
+// Inlined: a call from the softmax loop would spill that loop's live registers around
+// it (an out-of-line version measured about 5% slower).
 __device__ __forceinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, const WaitCtl ctl) {
   const uint64_t t0 = global_timer_ns();
   for (;;) {
@@ -142,21 +142,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Named barrier over `count` threads (a multiple of 32); id 0 is __syncthreads.
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// Per-warpgroup register reallocation (every warp of a warpgroup executes the same one).
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-
 // ---------------------------------------------------------------------------------
 // tcgen05: tensor memory allocation, MMA, commit, loads/stores, fences.
 // ---------------------------------------------------------------------------------
@@ -177,28 +162,6 @@ __device__ __forceinline__ void tc_fence_before() {
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// D(tmem) = A(smem) * B(smem)^T (+ D when accumulate != 0); kind::f16, one CTA.
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D(tmem) = A(tmem) * B(smem) (+ D when accumulate != 0); kind::f16, one CTA.
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 // A whole K loop of one 128 x 128 (or 128 x D) product in one asm block, so the issuing
@@ -235,86 +198,6 @@ __device__ __forceinline__ void mma_ss_kloop(uint32_t d_tmem, uint64_t a_desc, u
       "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
       "MMA_SS_DONE_%=:\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "n"(KSTEPS)
-      : "memory");
-}
-
-// The same SS K loop when A and B tiles have different row counts, so their 64-column
-// slabs sit a different distance apart: A slabs `A_SLAB` and B slabs `B_SLAB` descriptor
-// units (16 B) apart.  Used for S = Q K^T with 128-row Q tiles and 64-row K tiles.
-template <int KSTEPS, int A_SLAB, int B_SLAB>
-__device__ __forceinline__ void mma_ss_kloop_ab(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
-  static_assert(KSTEPS == 4 || KSTEPS == 8, "d = 64 or 128");
-  asm volatile(
-      "{\n\t.reg .pred pt, pf;\n\t.reg .b64 a, b;\n\t"
-      "setp.eq.u32 pt, 0, 0;\n\t"
-      "setp.ne.u32 pf, 0, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, pf;\n\t"
-      "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
-      "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
-      "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
-      ".reg .pred p8;\n\t"
-      "setp.eq.u32 p8, %4, 8;\n\t"
-      "@!p8 bra.uni MMA_SSAB_DONE_%=;\n\t"
-      "add.s64 a, %1, %5;\n\tadd.s64 b, %2, %9;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
-      "add.s64 a, %1, %6;\n\tadd.s64 b, %2, %10;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
-      "add.s64 a, %1, %7;\n\tadd.s64 b, %2, %11;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
-      "add.s64 a, %1, %8;\n\tadd.s64 b, %2, %12;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, pt;\n\t"
-      "MMA_SSAB_DONE_%=:\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "n"(KSTEPS), "n"(A_SLAB), "n"(A_SLAB + 2), "n"(A_SLAB + 4),
-      "n"(A_SLAB + 6), "n"(B_SLAB), "n"(B_SLAB + 2), "n"(B_SLAB + 4), "n"(B_SLAB + 6)
-      : "memory");
-}
-
-// TS form for O (+)= P V: A = P in TMEM (16 keys = 8 columns per step), B = V MN-major
-// (16 key rows of 128 B = 2048 B per step, +128 in descriptor units).  `accumulate`
-// applies to the first step only (0 for the first key tile of a query tile).
-__device__ __forceinline__ void mma_ts_kloop8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                              uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred pt, p0;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
-      "setp.eq.u32 pt, 0, 0;\n\t"
-      "setp.ne.b32 p0, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
-      "add.u32 a, %1, 8;\n\tadd.s64 b, %2, 128;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
-      "add.u32 a, %1, 16;\n\tadd.s64 b, %2, 256;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
-      "add.u32 a, %1, 24;\n\tadd.s64 b, %2, 384;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
-      "add.u32 a, %1, 32;\n\tadd.s64 b, %2, 512;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
-      "add.u32 a, %1, 40;\n\tadd.s64 b, %2, 640;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
-      "add.u32 a, %1, 48;\n\tadd.s64 b, %2, 768;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
-      "add.u32 a, %1, 56;\n\tadd.s64 b, %2, 896;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Half of that K loop: 4 steps (64 keys) from P column a_tmem and V descriptor b_desc.
-__device__ __forceinline__ void mma_ts_kloop4(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                              uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred pt, p0;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
-      "setp.eq.u32 pt, 0, 0;\n\t"
-      "setp.ne.b32 p0, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
-      "add.u32 a, %1, 8;\n\tadd.s64 b, %2, 128;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
-      "add.u32 a, %1, 16;\n\tadd.s64 b, %2, 256;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t"
-      "add.u32 a, %1, 24;\n\tadd.s64 b, %2, 384;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, pt;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -361,18 +244,6 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-}
-
-// 16 columns: the same, for roles that run with few registers.
-__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
 }
@@ -453,15 +324,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
       "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 
