@@ -15,9 +15,9 @@
 // and finally O_i / l (bf16) and LSE = m + ln l (fp32), each written to HBM once.  The
 // score matrix never leaves the SM.
 //
-// Pipeline.  The softmax reads its whole 128-score row of S from TMEM with one load and
-// says so at once; S of the next key tile can then be computed into the same TMEM
-// columns while the softmax is still exponentiating, so per query tile the tensor core
+// Pipeline.  The softmax reads its whole 128-score row of S from TMEM (two 64-column
+// loads, one wait) and says so at once; S of the next key tile can then be computed into
+// the same TMEM columns while the softmax is still exponentiating, so per query tile the tensor core
 // runs S_{j+1} in the shadow of softmax_j and P_j V_j right after it (P lives in shared
 // memory, one 32 KB buffer per query tile, in two 64-key slabs with their own barriers so
 // each half's P.V starts as soon as that half is stored).  The two query tiles run the
@@ -38,7 +38,14 @@
 //                of shared-memory slots); warps 9 and 10: one MMA-issuing thread per query
 //                tile (warp 9 also owns the TMEM allocation); warp 11 idle.
 // With 12 warps, at most 3 share an SM sub-partition, so each thread gets up to 168
-// registers: enough for a softmax thread to hold its whole 128-score row.
+// registers: enough for a softmax thread to hold its whole 128-score row.  There is no
+// separate correction warpgroup: with lazy rescaling (below) O is rescaled rarely, so the
+// softmax warps do it themselves.  A fourth warpgroup taking over the epilogue (512
+// threads, softmax re-sized to 192 registers with setmaxnreg) measured slower: it made
+// every key tile's softmax about 6% longer, more than the epilogue it removed.
+// Per key tile a softmax warp waits on two barriers (S ready, both halves of the previous
+// P read); each wait tests the phase without blocking first, since it has nearly always
+// completed already and every mbarrier test costs a shared-memory round trip.
 // Epilogue: O / l is written as bf16 into the query tile's P buffer (free once the last
 // P.V has completed) in the 128-byte-swizzled layout of the O tensor map and stored with
 // TMA, one 64-column slab per store.
