@@ -321,7 +321,7 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   if ((rc = make_map(&maps.v, v, B * Hkv, Nk, d, tc::BN)) != FA_OK) return rc;
   if (split)
     maps.o = maps.q;  // the split-KV epilogue writes fp32 partials without TMA
-  else if ((rc = make_map(&maps.o, o, B * Hq, Nq, d, tc::BM)) != FA_OK)
+  else if ((rc = make_map(&maps.o, o, B * Hq, Nq, d, 32)) != FA_OK)  // one box per warp's 32 rows
     return rc;
   tc::Params p;
   p.o = static_cast<__nv_bfloat16*>(o);

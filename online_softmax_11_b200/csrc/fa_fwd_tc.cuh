@@ -47,8 +47,9 @@
 // P read); each wait tests the phase without blocking first, since it has nearly always
 // completed already and every mbarrier test costs a shared-memory round trip.
 // Epilogue: O / l is written as bf16 into the query tile's P buffer (free once the last
-// P.V has completed) in the 128-byte-swizzled layout of the O tensor map and stored with
-// TMA, one 64-column slab per store.
+// P.V has completed) in the 128-byte-swizzled layout of the O tensor map, and each warp
+// stores its own 32 rows with TMA (boxes of 32 rows x 64 columns), waiting for the store
+// to have read them only when it next writes P there.
 //
 // Online-softmax details:
 //   * Scores are handled in log2 units, u = s * scale * log2(e), so P = exp2(u - m) is one
@@ -111,9 +112,7 @@ struct Layout {
   static constexpr int kBarPFull = kBarSFree + NQ;        // [NQ][2]: P of key half 0 / 1 stored
   static constexpr int kBarPFree = kBarPFull + 2 * NQ;    // [NQ][2]: ... and read by its P.V
   static constexpr int kBarOFull = kBarPFree + 2 * NQ;    // [NQ]
-  static constexpr int kBarStgFull = kBarOFull + NQ;      // [NQ]: O staged in shared memory
-  static constexpr int kBarStgEmpty = kBarStgFull + NQ;   // [NQ]: ... and read by its TMA store
-  static constexpr int kBarDrain = kBarStgEmpty + NQ;
+  static constexpr int kBarDrain = kBarOFull + NQ;
   static constexpr int kNumBars = kBarDrain + NQ;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // u32 tmem base, int abort flag
   static constexpr int kBytes = kMiscOff + 16;
@@ -473,8 +472,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars[L::kBarPFree + 2 * i + h], 1);
       }
       mbar_init(&bars[L::kBarOFull + i], 1);
-      mbar_init(&bars[L::kBarStgFull + i], BM);
-      mbar_init(&bars[L::kBarStgEmpty + i], 1);
     }
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&bars[L::kBarKvFull + s], 1);
@@ -661,7 +658,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t colO = L::col_o(i);
     uint8_t* prow = smem + L::kPOff + i * L::kPBytes + trow * 128;  // this row of P (slab 0)
     const int rsw = trow & 7;
-    uint32_t s_phase = 0, o_phase = 0, g = 0, stg_cnt = 0;
+    uint32_t s_phase = 0, o_phase = 0, g = 0;
+    bool stg_pending = false;  // this warp's last O store may still be reading its rows of P
 
     for_each_tile(p, [&](const WorkTile& w) {
       const TileRange& t = w.tr(i);
@@ -771,6 +769,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // shared-memory round trip, so the first half's release is not waited for.
           if (h == 0 && !__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarPFree + 2 * i + 1], (g & 1u) ^ 1u, ctl)))
             return false;
+          if (h == 0 && stg_pending) {  // these rows of P held O for the warp's last TMA store
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+            stg_pending = false;
+          }
           if constexpr (!kCap) {
             lt += make_p<PMode::kPlainMixed>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
           } else if (wtier == 0) {
@@ -854,10 +857,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       }
       // O / lr as bf16 into this query tile's P buffer (free: the last P.V, which read
-      // it, has completed) in the 128-byte-swizzled layout of the O tensor map, then one
-      // thread stores it with TMA, one 64-column slab per store; rows past Nq fall
-      // outside the tensor and are not written.  The buffer is P again once the stores
-      // have read it.
+      // it, has completed) in the 128-byte-swizzled layout of the O tensor map, then lane 0
+      // of each warp stores the warp's 32 rows with TMA, one 64-column slab per store, with
+      // no barrier across warps.  The warp waits for its stores to have read the rows only
+      // when it next writes P there (the first tile of the next work tile).
       uint32_t r[D];
       if (t.part) {
         if constexpr (D == 128)
@@ -879,26 +882,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                        pack_bf16x2(__uint_as_float(rq[6]) * inv, __uint_as_float(rq[7]) * inv));
       }
       fence_proxy_async_smem();
-      mbar_arrive(&bars[L::kBarStgFull + i]);
+      __syncwarp();  // the warp's rows are staged
+      // each warp stores its own 32 rows (a 32-row box per 64-column slab); a box that
+      // starts past Nq has nothing to write, one that ends past it is clipped
+      const int wrow = t.r0 + wq * 32;
+      if (lane == 0 && wrow < p.Nq) {
+        uint8_t* base = smem + L::kPOff + i * L::kPBytes + wq * 32 * 128;
+        for (int h = 0; h < L::kHalves; ++h) tma_store_3d(&tmO, base + h * L::kHalfBytes, h * 64, wrow, w.bh);
+        bulk_commit_group();
+      }
+      stg_pending = true;
       if (p.lse != nullptr && row < p.Nq)
         p.lse[static_cast<int64_t>(w.bh) * p.Nq + row] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
-      bool ok = true;
-      if (trow == 0) {
-        ok = mbar_wait(&bars[L::kBarStgFull + i], stg_cnt & 1u, ctl);
-        if (ok) {
-          uint8_t* base = smem + L::kPOff + i * L::kPBytes;
-          for (int h = 0; h < L::kHalves; ++h) tma_store_3d(&tmO, base + h * L::kHalfBytes, h * 64, t.r0, w.bh);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-          mbar_arrive(&bars[L::kBarStgEmpty + i]);
-        }
-      }
-      __syncwarp();
-      if (!__all_sync(0xffffffffu, ok && mbar_wait(&bars[L::kBarStgEmpty + i], stg_cnt & 1u, ctl))) return false;
-      ++stg_cnt;
       return true;
     });
-    if (trow == 0) bulk_wait_group0();  // the last O stores have completed
+    if (lane == 0) bulk_wait_group0();  // the last O stores have completed
   }
 
   // ---- teardown
