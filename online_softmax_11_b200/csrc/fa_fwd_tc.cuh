@@ -864,7 +864,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t r[D];
       if (t.part) {
         if constexpr (D == 128)
-          tmem_ld128_wait(lane_base + colO, r);
+          tmem_ld64x2_wait(lane_base + colO, r);
         else
           tmem_ld64_wait(lane_base + colO, r);
       } else {  // no key at all for this query tile (fewer keys than queries, causal)
