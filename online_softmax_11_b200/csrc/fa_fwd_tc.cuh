@@ -872,14 +872,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int x = 0; x < D; ++x) r[x] = 0u;
       }
       uint8_t* stg = smem + L::kPOff + i * L::kPBytes + trow * 128;
+      const float2 inv2 = make_float2(inv, inv);
+      auto scaled = [&](const uint32_t* rq) {  // two columns of O / lr, packed to bf16
+        const float2 v = __fmul2_rn(make_float2(__uint_as_float(rq[0]), __uint_as_float(rq[1])), inv2);
+        return pack_bf16x2(v.x, v.y);
+      };
 #pragma unroll
       for (int q = 0; q < D / 8; ++q) {  // 16-byte chunk q of the row: slab q / 8, chunk q % 8
         const uint32_t* rq = r + 8 * q;
         *reinterpret_cast<uint4*>(stg + (q >> 3) * L::kHalfBytes + (((q & 7) ^ rsw) << 4)) =
-            make_uint4(pack_bf16x2(__uint_as_float(rq[0]) * inv, __uint_as_float(rq[1]) * inv),
-                       pack_bf16x2(__uint_as_float(rq[2]) * inv, __uint_as_float(rq[3]) * inv),
-                       pack_bf16x2(__uint_as_float(rq[4]) * inv, __uint_as_float(rq[5]) * inv),
-                       pack_bf16x2(__uint_as_float(rq[6]) * inv, __uint_as_float(rq[7]) * inv));
+            make_uint4(scaled(rq), scaled(rq + 2), scaled(rq + 4), scaled(rq + 6));
       }
       fence_proxy_async_smem();
       __syncwarp();  // the warp's rows are staged
