@@ -17,10 +17,10 @@
 //
 // Pipeline.  The softmax reads its whole 128-score row of S from TMEM (two 64-column
 // loads, one wait) and says so at once; S of the next key tile can then be computed into
-// the same TMEM columns while the softmax is still exponentiating, so per query tile the tensor core
-// runs S_{j+1} in the shadow of softmax_j and P_j V_j right after it (P lives in shared
-// memory, one 32 KB buffer per query tile, in two 64-key slabs with their own barriers so
-// each half's P.V starts as soon as that half is stored).  The two query tiles run the
+// the same TMEM columns while the softmax is still exponentiating, so per query tile the
+// tensor core runs S_{j+1} in the shadow of softmax_j and P_j V_j right after it (P lives
+// in shared memory, one 32 KB buffer per query tile, in two 64-key slabs with their own
+// barriers so each half's P.V starts as soon as that half is stored).  The two query tiles run the
 // same chain independently and share the tensor core and the K/V ring.  The ring streams
 // K one tile ahead of V (K_0, K_1, V_0, K_2, V_1, ...), the order the MMAs consume them.
 //
@@ -748,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
 
         // P = exp2(u - m) per 64-key half into its shared-memory slab, once the previous
-        // tile's P.V half has read the slab.  lt: fp32 sum of this tile's P; pmax: the P of
+        // tile's P.V has read the slabs.  lt: fp32 sum of this tile's P; pmax: the P of
         // the tile maximum, recomputed with the same instructions as in make_p (so it is
         // bit-identical to the value packed).
         float lt = 0.f, pmax;
@@ -760,99 +760,85 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if constexpr (!kCap) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float* sh = s + h * kHalf;
-          uint8_t* ph = prow + h * L::kHalfBytes;
-          // the previous tile's P.V has read both slabs: one wait, on the second half's
-          // release, covers both, since the MMAs of one thread complete in the order they
-          // were issued (the first wait of a fresh barrier passes: there is no previous
-          // tile).  It has nearly always come by now, and every mbarrier test costs a
-          // shared-memory round trip, so the first half's release is not waited for.
-          if (h == 0 && !__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarPFree + 2 * i + 1], (g & 1u) ^ 1u, ctl)))
-            return false;
-          if (h == 0 && stg_pending) {  // these rows of P held O for the warp's last TMA store
-            if (lane == 0) bulk_wait_group_read0();
-            __syncwarp();
-            stg_pending = false;
-          }
-          if constexpr (!kCap) {
-            lt += make_p<PMode::kPlainMixed>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
-          } else if (wtier == 0) {
-            lt += make_p<PMode::kCapShort>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
-          } else if (wtier == 1) {
-            lt += make_p<PMode::kCapLong>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
-          } else {
-            lt += make_p<PMode::kCapGeneral>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
-          }
-          fence_proxy_async_smem();  // the tensor core reads P through the async proxy
-          if (h == 0 && rescale) {
-            // O must hold the previous tile's whole P.V: its second half has landed, as the
-            // wait above has shown
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t r[32];
-              tmem_ld32_wait(lane_base + colO + c * 32, r);
-#pragma unroll
-              for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-              tmem_st32(lane_base + colO + c * 32, r);
+          for (int h = 0; h < 2; ++h) {
+            const float* sh = s + h * kHalf;
+            uint8_t* ph = prow + h * L::kHalfBytes;
+            // the previous tile's P.V has read both slabs: one wait, on the second half's
+            // release, covers both, since the MMAs of one thread complete in the order they
+            // were issued (the first wait of a fresh barrier passes: there is no previous
+            // tile).  It has nearly always come by now, and every mbarrier test costs a
+            // shared-memory round trip, so the first half's release is not waited for.
+            if (h == 0 && !__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarPFree + 2 * i + 1], (g & 1u) ^ 1u, ctl)))
+              return false;
+            if (h == 0 && stg_pending) {  // these rows of P held O for the warp's last TMA store
+              if (lane == 0) bulk_wait_group_read0();
+              __syncwarp();
+              stg_pending = false;
             }
-            tmem_wait_st();
+            lt += make_p<PMode::kPlainMixed>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
+            fence_proxy_async_smem();  // the tensor core reads P through the async proxy
+            if (h == 0 && rescale) {
+              // O must hold the previous tile's whole P.V: its second half has landed, as the
+              // wait above has shown
+              tc_fence_after();
+#pragma unroll 1
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32_wait(lane_base + colO + c * 32, r);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+                tmem_st32(lane_base + colO + c * 32, r);
+              }
+              tmem_wait_st();
+            }
+            // this half of P is stored (and O rescaled): its P.V can start
+            tc_fence_before();
+            mbar_arrive(&bars[L::kBarPFull + 2 * i + h]);
           }
-          // this half of P is stored (and O rescaled): its P.V can start
-          tc_fence_before();
-          mbar_arrive(&bars[L::kBarPFull + 2 * i + h]);
-        }
         } else {
-        // Soft-capped launches run both halves through one loop body: their three P tiers
-        // are long code, and the smaller loop measured faster (+8 % on the window +
-        // soft-cap workloads); the plain launch keeps the unrolled form.
+          // Soft-capped launches run both halves through one loop body: their three P tiers
+          // are long code, and the smaller loop measured faster (+8 % on the window +
+          // soft-cap workloads); the plain launch keeps the unrolled form.
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          const float* sh = s;  // the half being converted is always in s[0 .. 63]
-          uint8_t* ph = prow + h * L::kHalfBytes;
-          // the previous tile's P.V has read both slabs: one wait, on the second half's
-          // release, covers both, since the MMAs of one thread complete in the order they
-          // were issued (the first wait of a fresh barrier passes: there is no previous
-          // tile).  It has nearly always come by now, and every mbarrier test costs a
-          // shared-memory round trip, so the first half's release is not waited for.
-          if (h == 0 && !__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarPFree + 2 * i + 1], (g & 1u) ^ 1u, ctl)))
-            return false;
-          if (h == 0 && stg_pending) {  // these rows of P held O for the warp's last TMA store
-            if (lane == 0) bulk_wait_group_read0();
-            __syncwarp();
-            stg_pending = false;
-          }
-          if constexpr (!kCap) {
-            lt += make_p<PMode::kPlainMixed>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
-          } else if (wtier == 0) {
-            lt += make_p<PMode::kCapShort>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
-          } else if (wtier == 1) {
-            lt += make_p<PMode::kCapLong>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
-          } else {
-            lt += make_p<PMode::kCapGeneral>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
-          }
-          fence_proxy_async_smem();  // the tensor core reads P through the async proxy
-          if (h == 0 && rescale) {
-            // O must hold the previous tile's whole P.V: its second half has landed, as the
-            // wait above has shown
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t r[32];
-              tmem_ld32_wait(lane_base + colO + c * 32, r);
-#pragma unroll
-              for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-              tmem_st32(lane_base + colO + c * 32, r);
+          for (int h = 0; h < 2; ++h) {
+            const float* sh = s;  // the half being converted is always in s[0 .. 63]
+            uint8_t* ph = prow + h * L::kHalfBytes;
+            // as above: one wait for both slabs of the previous tile's P
+            if (h == 0 && !__all_sync(0xffffffffu, mbar_wait(&bars[L::kBarPFree + 2 * i + 1], (g & 1u) ^ 1u, ctl)))
+              return false;
+            if (h == 0 && stg_pending) {  // these rows of P held O for the warp's last TMA store
+              if (lane == 0) bulk_wait_group_read0();
+              __syncwarp();
+              stg_pending = false;
             }
-            tmem_wait_st();
-          }
-          // this half of P is stored (and O rescaled): its P.V can start
-          tc_fence_before();
-          mbar_arrive(&bars[L::kBarPFull + 2 * i + h]);
+            if (wtier == 0) {
+              lt += make_p<PMode::kCapShort>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
+            } else if (wtier == 1) {
+              lt += make_p<PMode::kCapLong>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
+            } else {
+              lt += make_p<PMode::kCapGeneral>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
+            }
+            fence_proxy_async_smem();  // the tensor core reads P through the async proxy
+            if (h == 0 && rescale) {
+              // O must hold the previous tile's whole P.V: its second half has landed, as the
+              // wait above has shown
+              tc_fence_after();
+#pragma unroll 1
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32_wait(lane_base + colO + c * 32, r);
 #pragma unroll
-          for (int c = 0; c < kHalf; ++c) s[c] = s[c + kHalf];  // the second half moves down
-        }
+                for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+                tmem_st32(lane_base + colO + c * 32, r);
+              }
+              tmem_wait_st();
+            }
+            // this half of P is stored (and O rescaled): its P.V can start
+            tc_fence_before();
+            mbar_arrive(&bars[L::kBarPFull + 2 * i + h]);
+#pragma unroll
+            for (int c = 0; c < kHalf; ++c) s[c] = s[c + kHalf];  // the second half moves down
+          }
         }
         ++g;
         if constexpr (!kCap) {
