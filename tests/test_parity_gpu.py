@@ -133,6 +133,8 @@ BF16_CASES = [
     (1, 2, 2, 520, 64, False, 0, 50.0, 1.0),     # |s scale / cap| < 0.12: short series
     (1, 2, 2, 600, 128, True, 0, 0.0, 8.0),      # large logits: running max moves a lot
     (1, 2, 2, 600, 64, False, 0, 0.0, 8.0),
+    (1, 2, 2, 700, 128, True, 0, 50.0, 8.0),     # soft-cap with a moving maximum: O rescaled
+    (1, 2, 1, 650, 64, True, 300, 30.0, 8.0),    # ... with a window, GQA and d = 64
 ]
 
 
