@@ -170,30 +170,6 @@ __device__ __forceinline__ float tanh_cap(float x) {
   return copysignf(t, x);
 }
 
-// 2^x for a pair of floats on the FMA pipe instead of the exponential unit.  x is split
-// as n + f with n = round(x) (the 1.5 * 2^23 shifter: after x + M the low mantissa bits
-// of the sum hold n), 2^f on [-1/2, 1/2] is a cubic, and n is added to the exponent
-// field.  The cubic's coefficients were fitted for minimum relative error on
-// [-1/2, 1/2] (Lawson's iteratively reweighted least squares): max relative error
-// 7.5e-5, below the 2^-9 of the bf16 rounding that P goes through next.  x is clamped at
-// -125 so the exponent cannot underflow, and anything below -125 (a masked key's -inf
-// included) gives exactly 0, as the exponential unit does for -inf; between 2^-125 and
-// the unit's own underflow the two differ by less than anything that can matter.
-__device__ __forceinline__ float2 exp2_fma_pair(float2 x) {
-  const bool zx = x.x < -125.0f, zy = x.y < -125.0f;
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 shifter = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
-  const float2 r = __fadd2_rn(x, shifter);
-  const float2 n = __fadd2_rn(r, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);  // x - n, exact
-  float2 q = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.2426111400f, 0.2426111400f));
-  q = __ffma2_rn(q, f, make_float2(0.6932609677f, 0.6932609677f));
-  q = __ffma2_rn(q, f, make_float2(0.9999280572f, 0.9999280572f));
-  return make_float2(zx ? 0.f : __uint_as_float(__float_as_uint(q.x) + (__float_as_uint(r.x) << 23)),
-                     zy ? 0.f : __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(r.y) << 23)));
-}
-
 __device__ __forceinline__ float2 ex2_pair(float2 x) { return make_float2(ex2_approx(x.x), ex2_approx(x.y)); }
 
 // tanh for a pair known to satisfy |x| < 0.3 (Taylor terms through x^11), or |x| < 0.12
@@ -217,9 +193,9 @@ __device__ __forceinline__ float2 tanh_small_pair(float2 x) {
 
 // How P is produced from the scores of one tile (chosen per tile, warp-uniformly).
 enum class PMode {
-  kPlainMixed,   // no soft-cap: 3 of 4 pairs on ex2, 1 of 4 on the FMA pipe (masked keys,
-                 // -inf, give exactly 0 on both); one code path for masked and unmasked
-                 // tiles keeps the loop small
+  kPlain,        // no soft-cap: ex2 on the exponential unit for every score (masked keys,
+                 // -inf, give exactly 0); one code path for masked and unmasked tiles
+                 // keeps the loop small
   kCapShort,     // soft-cap, every |s * scale / cap| < 0.12
   kCapLong,      // soft-cap, every |s * scale / cap| < 0.3
   kCapGeneral,   // soft-cap, anything else (including masked keys)
@@ -243,12 +219,8 @@ __device__ __forceinline__ float make_p(const float* s, uint8_t* prow, int rsw, 
     for (int x = 0; x < 4; ++x) {
       const float2 sv = make_float2(s[c * 8 + 2 * x], s[c * 8 + 2 * x + 1]);
       float2 e;
-      if constexpr (kMode == PMode::kPlainMixed) {
-        const float2 u = __ffma2_rn(sv, make_float2(scale_log2, scale_log2), negm);
-        if (kMode == PMode::kPlainMixed && x == 3)  // one pair in four on the FMA pipe
-          e = exp2_fma_pair(u);
-        else
-          e = ex2_pair(u);
+      if constexpr (kMode == PMode::kPlain) {
+        e = ex2_pair(__ffma2_rn(sv, make_float2(scale_log2, scale_log2), negm));
       } else if constexpr (kMode == PMode::kCapShort || kMode == PMode::kCapLong) {
         const float2 t = tanh_small_pair<kMode == PMode::kCapShort>(__fmul2_rn(sv, make_float2(cap_inner, cap_inner)));
         e = ex2_pair(__ffma2_rn(t, make_float2(cap_outer, cap_outer), negm));
@@ -694,23 +666,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h_hi = w_lo;
 
         // The whole row of S in registers with one TMEM round trip, then the row maximum (and
-        // minimum, for the soft-cap range check) with three-input max: three chains over
-        // the columns whose exp2 runs on the MUFU in plain (no soft-cap) tiles, one over those
-        // on the FMA pipe (pair 3 of every 4, i.e. columns 8k+6, 8k+7), so the tile
-        // maximum's P can be recomputed with the very arithmetic that produced it.
+        // minimum, for the soft-cap range check) with three-input max in four independent
+        // chains.
         float s[BN];
         load_row<kSinks>(lane_base + colS, need_mask, sink_cols, h_lo, h_hi, c_hi, s);
         // S is in registers: the next key tile's S may overwrite it
         tc_fence_before();
         mbar_arrive(&bars[L::kBarSFree + i]);
-        float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F, mx2 = -CUDART_INF_F, mx_emu = -CUDART_INF_F;
+        float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F, mx2 = -CUDART_INF_F, mx3 = -CUDART_INF_F;
         float mn0 = CUDART_INF_F, mn1 = CUDART_INF_F;
 #pragma unroll
         for (int c = 0; c < BN; c += 8) {
           mx0 = fmax3(mx0, s[c], s[c + 1]);
           mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
           mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
-          mx_emu = fmax3(mx_emu, s[c + 6], s[c + 7]);
+          mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
         }
         if constexpr (kCap) {
 #pragma unroll
@@ -719,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mn1 = fmin3(mn1, s[c + 2], s[c + 3]);
           }
         }
-        const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx_emu));
+        const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
         const float mn = fminf(mn0, mn1);
         float m_tile;
         if constexpr (kCap)
@@ -775,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               __syncwarp();
               stg_pending = false;
             }
-            lt += make_p<PMode::kPlainMixed>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
+            lt += make_p<PMode::kPlain>(sh, ph, rsw, p.scale_log2, 0.f, 0.f, m_use);
             fence_proxy_async_smem();  // the tensor core reads P through the async proxy
             if (h == 0 && rescale) {
               // O must hold the previous tile's whole P.V: its second half has landed, as the
@@ -843,7 +813,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++g;
         if constexpr (!kCap) {
           const float u = fmaf(mx, p.scale_log2, -m_use);
-          pmax = (mx_emu == mx) ? exp2_fma_pair(make_float2(u, u)).x : ex2_approx(u);
+          pmax = ex2_approx(u);
         } else {
           const float xm = mx * p.cap_inner;
           if (wtier == 0)
