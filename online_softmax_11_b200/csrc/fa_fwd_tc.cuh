@@ -172,23 +172,25 @@ __device__ __forceinline__ float tanh_cap(float x) {
 
 __device__ __forceinline__ float2 ex2_pair(float2 x) { return make_float2(ex2_approx(x.x), ex2_approx(x.y)); }
 
-// tanh for a pair known to satisfy |x| < 0.3 (Taylor terms through x^11), or |x| < 0.12
-// when kShort (terms through x^7; the next term is below 1e-10 there).
+// u = co tanh(x) - m for a pair with |x| < 0.3: the Taylor series of tanh through x^11, or
+// through x^7 when kShort and |x| < 0.12 (the next term is below 1e-10 there), with the
+// outer scale co folded into its coefficients: co tanh(x) = x (co + x^2 (b1 + x^2 (b2 +
+// ...))), b_k = co c_k, c_k = -1/3, 2/15, -17/315, 62/2835, -1382/155925.  b holds b1 ..
+// b5 (kShort reads b1 .. b3).
 template <bool kShort>
-__device__ __forceinline__ float2 tanh_small_pair(float2 x) {
+__device__ __forceinline__ float2 cap_u_pair(float2 x, const float* b, float co, float2 negm) {
   const float2 x2 = __fmul2_rn(x, x);
-  float2 p;
+  float2 r;
   if (kShort) {
-    p = __ffma2_rn(make_float2(-17.0f / 315.0f, -17.0f / 315.0f), x2, make_float2(2.0f / 15.0f, 2.0f / 15.0f));
+    r = __ffma2_rn(make_float2(b[2], b[2]), x2, make_float2(b[1], b[1]));
   } else {
-    p = __ffma2_rn(make_float2(-1382.0f / 155925.0f, -1382.0f / 155925.0f), x2,
-                   make_float2(62.0f / 2835.0f, 62.0f / 2835.0f));
-    p = __ffma2_rn(p, x2, make_float2(-17.0f / 315.0f, -17.0f / 315.0f));
-    p = __ffma2_rn(p, x2, make_float2(2.0f / 15.0f, 2.0f / 15.0f));
+    r = __ffma2_rn(make_float2(b[4], b[4]), x2, make_float2(b[3], b[3]));
+    r = __ffma2_rn(r, x2, make_float2(b[2], b[2]));
+    r = __ffma2_rn(r, x2, make_float2(b[1], b[1]));
   }
-  p = __ffma2_rn(p, x2, make_float2(-1.0f / 3.0f, -1.0f / 3.0f));
-  p = __fmul2_rn(p, x2);
-  return __ffma2_rn(p, x, x);
+  r = __ffma2_rn(r, x2, make_float2(b[0], b[0]));
+  const float2 w = __ffma2_rn(r, x2, make_float2(co, co));
+  return __ffma2_rn(w, x, negm);
 }
 
 // How P is produced from the scores of one tile (chosen per tile, warp-uniformly).
@@ -209,7 +211,7 @@ constexpr int kHalf = BN / 2;  // the softmax works on 64-score halves of a row
 // operands in.  Returns the fp32 sum of these P.
 template <PMode kMode>
 __device__ __forceinline__ float make_p(const float* s, uint8_t* prow, int rsw, float scale_log2, float cap_inner,
-                                        float cap_outer, float m_use) {
+                                        float cap_outer, float m_use, const float* cap_b = nullptr) {
   const float2 negm = make_float2(-m_use, -m_use);
   float2 lsum0 = make_float2(0.f, 0.f), lsum1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -222,8 +224,8 @@ __device__ __forceinline__ float make_p(const float* s, uint8_t* prow, int rsw, 
       if constexpr (kMode == PMode::kPlain) {
         e = ex2_pair(__ffma2_rn(sv, make_float2(scale_log2, scale_log2), negm));
       } else if constexpr (kMode == PMode::kCapShort || kMode == PMode::kCapLong) {
-        const float2 t = tanh_small_pair<kMode == PMode::kCapShort>(__fmul2_rn(sv, make_float2(cap_inner, cap_inner)));
-        e = ex2_pair(__ffma2_rn(t, make_float2(cap_outer, cap_outer), negm));
+        e = ex2_pair(cap_u_pair<kMode == PMode::kCapShort>(__fmul2_rn(sv, make_float2(cap_inner, cap_inner)),
+                                                           cap_b, cap_outer, negm));
       } else {
         e.x = ex2_approx(fmaf(tanh_cap(sv.x * cap_inner), cap_outer, -m_use));
         e.y = ex2_approx(fmaf(tanh_cap(sv.y * cap_inner), cap_outer, -m_use));
@@ -632,6 +634,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rsw = trow & 7;
     uint32_t s_phase = 0, o_phase = 0, g = 0;
     bool stg_pending = false;  // this warp's last O store may still be reading its rows of P
+    // soft-cap series coefficients with the outer scale folded in (tanh's Taylor terms)
+    const float cap_b[5] = {p.cap_outer * (-1.0f / 3.0f), p.cap_outer * (2.0f / 15.0f), p.cap_outer * (-17.0f / 315.0f),
+                            p.cap_outer * (62.0f / 2835.0f), p.cap_outer * (-1382.0f / 155925.0f)};
 
     for_each_tile(p, [&](const WorkTile& w) {
       const TileRange& t = w.tr(i);
@@ -782,9 +787,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               stg_pending = false;
             }
             if (wtier == 0) {
-              lt += make_p<PMode::kCapShort>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
+              lt += make_p<PMode::kCapShort>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use, cap_b);
             } else if (wtier == 1) {
-              lt += make_p<PMode::kCapLong>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
+              lt += make_p<PMode::kCapLong>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use, cap_b);
             } else {
               lt += make_p<PMode::kCapGeneral>(sh, ph, rsw, 0.f, p.cap_inner, p.cap_outer, m_use);
             }
@@ -817,9 +822,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const float xm = mx * p.cap_inner;
           if (wtier == 0)
-            pmax = ex2_approx(fmaf(tanh_small_pair<true>(make_float2(xm, xm)).x, p.cap_outer, -m_use));
+            pmax = ex2_approx(cap_u_pair<true>(make_float2(xm, xm), cap_b, p.cap_outer, make_float2(-m_use, -m_use)).x);
           else if (wtier == 1)
-            pmax = ex2_approx(fmaf(tanh_small_pair<false>(make_float2(xm, xm)).x, p.cap_outer, -m_use));
+            pmax = ex2_approx(cap_u_pair<false>(make_float2(xm, xm), cap_b, p.cap_outer, make_float2(-m_use, -m_use)).x);
           else
             pmax = ex2_approx(fmaf(tanh_cap(xm), p.cap_outer, -m_use));
         }
