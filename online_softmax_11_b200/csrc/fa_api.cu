@@ -46,10 +46,10 @@ int current_device(int* dev) {
   return FA_OK;
 }
 
-// Shared-memory size, and a check of the launch register count: the kernel re-splits its
-// registers between warpgroups with setmaxnreg, and the shares add up to exactly
-// kThreads x kLaunchRegs.  A build whose launch count differs would leave a register
-// request unsatisfiable, so such a kernel is refused here instead of launched.
+// Shared-memory size, and a check of the launch register count: one CTA of kThreads
+// threads must fit an SM's register file at kLaunchRegs registers each.  A build that
+// uses more (or allows fewer threads per block) could not launch, so such a kernel is
+// refused here instead.
 template <typename K>
 cudaError_t prepare_tc_kernel(K kernel, int smem_bytes, bool* regs_ok) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
